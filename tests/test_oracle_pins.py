@@ -1,0 +1,334 @@
+"""Pins for the CPU oracle, against things other than the oracle itself.
+
+Each check is written as a function of a GEMM callable so that the same
+checks can be run against deliberately broken copies of the oracle (the
+"planted mistakes" at the bottom): every plausible mistake must fail at least
+one pin.  All of this runs on the CPU.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tlg_workloads as wl
+from conftest import read_golden_blocks, read_golden_pairs
+
+
+def f16(x):
+    return np.asarray(x, dtype=np.float16)
+
+
+def dec(x):
+    return np.asarray(x, dtype=np.float16).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------- codec
+
+def test_decode_exhaustive_matches_numpy():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.f16_decode(bits)
+    want = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))
+
+
+def test_decode_golden_values():
+    for h, v in read_golden_pairs("f16_values.txt"):
+        got = oracle.f16_decode(np.array([int(h, 16)], dtype=np.uint16))[0]
+        want = float(v)
+        assert got == want, (h, got, want)
+        assert math.copysign(1.0, got) == math.copysign(1.0, want), h
+
+
+def test_encode_golden_rounding():
+    for x, h in read_golden_pairs("f16_rounding.txt"):
+        got = int(oracle.f16_encode_rne(np.array([float(x)]))[0])
+        assert got == int(h, 16), (x, hex(got), h)
+
+
+def test_encode_roundtrips_every_finite_fp16():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = bits.view(np.float16).astype(np.float64)
+    finite = np.isfinite(vals)
+    back = oracle.f16_encode_rne(vals[finite])
+    assert np.array_equal(back, bits[finite])
+
+
+def test_encode_matches_numpy_on_random_doubles():
+    rng = np.random.default_rng(123)
+    x = np.concatenate([
+        rng.standard_normal(200000) * 10.0 ** rng.integers(-9, 6, 200000),
+        rng.uniform(-70000, 70000, 50000),
+        # exact midpoints between neighbouring fp16 values
+        (np.arange(0, 31743, 7, dtype=np.uint16).view(np.float16).astype(np.float64)
+         + np.arange(1, 31744, 7, dtype=np.uint16).view(np.float16).astype(np.float64)) / 2,
+    ])
+    with np.errstate(over="ignore"):
+        want = x.astype(np.float16).view(np.uint16)
+    got = oracle.f16_encode_rne(x)
+    assert np.array_equal(got, want)
+
+
+# ----------------------------------------------------------------------------- pins as functions of a GEMM
+
+def pin_golden(gemm):
+    for ex in read_golden_blocks("gemm_worked_examples.txt"):
+        M, N, K = ex["shape"]
+        A = f16(ex["A"]).reshape(M, K)
+        B = f16(ex["B"]).reshape(K, N)
+        C = np.array(ex["C"]).reshape(M, N)
+        assert np.array_equal(gemm(A, B, None, False), C), ex["name"]
+
+
+def pin_golden_bias_relu(gemm):
+    for ex in read_golden_blocks("bias_relu_worked_examples.txt"):
+        M, N, K = ex["shape"]
+        A = f16(ex["A"]).reshape(M, K)
+        B = f16(ex["B"]).reshape(K, N)
+        bias = f16(ex["bias"])
+        C = np.array(ex["C"]).reshape(M, N)
+        assert np.array_equal(gemm(A, B, bias, True), C), ex["name"]
+
+
+def pin_identity(gemm):
+    rng = np.random.default_rng(1)
+    B = f16(rng.uniform(-1, 1, (37, 23)))
+    I = np.eye(37, dtype=np.float16)
+    assert np.array_equal(gemm(I, B, None, False), dec(B))
+    A = f16(rng.uniform(-1, 1, (19, 23)))
+    I2 = np.eye(23, dtype=np.float16)
+    assert np.array_equal(gemm(A, I2, None, False), dec(A))
+
+
+def pin_all_ones(gemm):
+    for M, N, K in [(3, 5, 1), (4, 7, 17), (2, 3, 256), (5, 2, 1000)]:
+        C = gemm(np.ones((M, K), np.float16), np.ones((K, N), np.float16), None, False)
+        assert np.array_equal(C, np.full((M, N), float(K)))
+
+
+def pin_numpy_matmul(gemm):
+    rng = np.random.default_rng(2)
+    for M, N, K in [(67, 45, 129), (1, 130, 257), (33, 1, 64)]:
+        A = f16(rng.uniform(-1, 1, (M, K)))
+        B = f16(rng.standard_normal((K, N)))
+        want = dec(A) @ dec(B)
+        scale = np.abs(dec(A)) @ np.abs(dec(B))
+        got = gemm(A, B, None, False)
+        assert np.all(np.abs(got - want) <= 1e-12 * (scale + 1e-300)), (M, N, K)
+
+
+def pin_fsum_dots(gemm):
+    rng = np.random.default_rng(3)
+    for K in [1, 2, 63, 64, 65, 1000]:
+        a = f16(rng.uniform(-1, 1, (1, K)))
+        b = f16(rng.uniform(-1, 1, (K, 1)))
+        exact = math.fsum(float(x) * float(y) for x, y in zip(dec(a)[0], dec(b)[:, 0]))
+        got = gemm(a, b, None, False)[0, 0]
+        bound = 1e-13 * math.fsum(abs(float(x) * float(y)) for x, y in zip(dec(a)[0], dec(b)[:, 0]))
+        assert abs(got - exact) <= bound, K
+
+
+def pin_transpose(gemm):
+    rng = np.random.default_rng(4)
+    A = f16(rng.uniform(-1, 1, (9, 13)))
+    B = f16(rng.uniform(-1, 1, (13, 6)))
+    assert np.array_equal(gemm(A, B, None, False).T, gemm(B.T.copy(), A.T.copy(), None, False))
+
+
+def pin_bias_column_broadcast(gemm):
+    rng = np.random.default_rng(5)
+    M, N, K = 6, 11, 4
+    bias = f16(rng.uniform(-0.5, 0.5, N))
+    zero = gemm(np.zeros((M, K), np.float16), f16(rng.uniform(-1, 1, (K, N))), bias, True)
+    assert np.array_equal(zero, np.tile(np.maximum(dec(bias), 0.0), (M, 1)))
+    neg = gemm(f16(rng.uniform(-1, 1, (M, K))), f16(rng.uniform(-1, 1, (K, N))),
+               np.full(N, -1000, np.float16), True)
+    assert np.array_equal(neg, np.zeros((M, N)))
+    A = f16(rng.uniform(-1, 1, (M, K)))
+    B = f16(rng.uniform(-1, 1, (K, N)))
+    r = gemm(A, B, bias, True)
+    assert np.all(r >= 0)
+    plain = gemm(A, B, None, False)
+    assert np.array_equal(r, np.maximum(plain + dec(bias)[None, :], 0.0))
+
+
+PINS = [pin_golden, pin_golden_bias_relu, pin_identity, pin_all_ones, pin_numpy_matmul,
+        pin_fsum_dots, pin_transpose, pin_bias_column_broadcast]
+
+
+def oracle_gemm(A, B, bias, relu):
+    return oracle.gemm(A, B, bias=bias, relu=relu, threads=2)
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
+def test_oracle_pins(pin):
+    pin(oracle_gemm)
+
+
+# ----------------------------------------------------------------------------- other invariants
+
+def test_sampled_equals_full_bit_for_bit():
+    A, B, bias = wl.make_operands(70, 90, 300, "uniform", bias=True, seed=7)
+    full = oracle.gemm(A, B, bias=bias, relu=True)
+    rows, cols = wl.sample_positions(70, 90, 500, seed=8)
+    at = oracle.gemm_at(A, B, rows.numpy(), cols.numpy(), bias=bias, relu=True)
+    assert np.array_equal(at, full[rows.numpy(), cols.numpy()])
+
+
+def test_thread_count_does_not_change_result():
+    A, B, _ = wl.make_operands(64, 48, 200, "normal025", seed=9)
+    r1 = oracle.gemm(A, B, threads=1)
+    r8 = oracle.gemm(A, B, threads=8)
+    assert np.array_equal(r1, r8)
+
+
+def test_pure_python_loop_agrees_on_tiny_input():
+    A, B, bias = wl.make_operands(3, 4, 5, "uniform", bias=True, seed=10)
+    a, b, bb = dec(A.numpy()), dec(B.numpy()), dec(bias.numpy())
+    want = np.zeros((3, 4))
+    for i in range(3):
+        for j in range(4):
+            s = 0.0
+            for k in range(5):
+                s += a[i, k] * b[k, j]
+            want[i, j] = max(s + bb[j], 0.0)
+    assert np.array_equal(oracle.gemm(A, B, bias=bias, relu=True), want)
+
+
+def test_empty_and_degenerate_shapes():
+    A = np.zeros((0, 5), np.float16)
+    B = np.ones((5, 3), np.float16)
+    assert oracle.gemm(A, B).shape == (0, 3)
+    A = np.zeros((4, 0), np.float16)
+    B = np.zeros((0, 3), np.float16)
+    assert np.array_equal(oracle.gemm(A, B), np.zeros((4, 3)))  # empty sum is 0
+    bias = f16([-1, 0.5, 2])
+    assert np.array_equal(oracle.gemm(A, B, bias=bias, relu=True), np.tile([0.0, 0.5, 2.0], (4, 1)))
+
+
+def test_uniform_generator_statistics():
+    # U[-1,1] entries: each product has variance 1/9, so an output has variance K/9 and mean 0.
+    w = wl.WORKLOADS["gemm_256_f32"]
+    A, B, _ = wl.workload_operands(w)
+    C = oracle.gemm(A, B)
+    K = w.K
+    assert abs(C.mean()) < 0.05 * math.sqrt(K / 9)
+    assert abs(C.var() / (K / 9) - 1.0) < 0.05
+    a = dec(A.numpy())
+    assert a.min() >= -1 and a.max() <= 1 and abs(a.var() - 1 / 3) < 0.01
+
+
+def test_inputs_are_seeded_and_ordered():
+    A1, B1, b1 = wl.make_operands(8, 9, 10, "uniform", bias=True, seed=0)
+    A2, B2, b2 = wl.make_operands(8, 9, 10, "uniform", bias=True, seed=0)
+    assert torch.equal(A1, A2) and torch.equal(B1, B2) and torch.equal(b1, b2)
+    g = torch.Generator().manual_seed(0)
+    assert torch.equal(A1, (torch.rand((8, 10), generator=g) * 2 - 1).half())
+    A3, _, _ = wl.make_operands(8, 9, 10, "uniform", seed=1)
+    assert not torch.equal(A1, A3)
+
+
+def test_tolerance_helper():
+    ref = np.array([0.0, 1.0, 100.0])
+    ok, worst, _ = oracle.within_tolerance(ref + np.array([0.009, 0.011, 0.2]), ref, "f32")
+    assert ok and worst < 1.0
+    ok, _, idx = oracle.within_tolerance(ref + np.array([0.0, 0.0, 0.3]), ref, "f32")
+    assert not ok and idx == (2,)
+    ok, _, _ = oracle.within_tolerance(np.array([np.nan, 1.0, 100.0]), ref, "f32")
+    assert not ok
+
+
+# ----------------------------------------------------------------------------- planted mistakes
+# Broken copies of the oracle's arithmetic (numpy, on the CPU).  Each must fail
+# at least one of the pins above, which shows the pins can see that mistake.
+
+def _ref(A, B, bias, relu):
+    C = dec(A) @ dec(B)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    if relu:
+        C = np.maximum(C, 0.0)
+    return C
+
+
+def mutant_dropped_last_k(A, B, bias, relu):
+    return _ref(np.ascontiguousarray(A[:, :-1]), np.ascontiguousarray(B[:-1, :]), bias, relu)
+
+
+def mutant_transposed_B(A, B, bias, relu):
+    K, N = B.shape
+    if K == N:
+        return _ref(A, np.ascontiguousarray(B.T), bias, relu)
+    return _ref(A, np.ascontiguousarray(B.reshape(N, K).T), bias, relu)
+
+
+def mutant_row_bias(A, B, bias, relu):
+    C = dec(A) @ dec(B)
+    if bias is not None:
+        M = C.shape[0]
+        bb = dec(bias)
+        C = C + np.resize(bb, M)[:, None]
+    return np.maximum(C, 0.0) if relu else C
+
+
+def mutant_bias_sign(A, B, bias, relu):
+    return _ref(A, B, None if bias is None else (-dec(bias)).astype(np.float16), relu)
+
+
+def mutant_relu_before_bias(A, B, bias, relu):
+    C = dec(A) @ dec(B)
+    if relu:
+        C = np.maximum(C, 0.0)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    return C
+
+
+def mutant_fp16_accumulator(A, B, bias, relu):
+    a, b = dec(A), dec(B)
+    M, K = a.shape
+    N = b.shape[1]
+    C = np.zeros((M, N), np.float16)
+    for k in range(K):
+        C = (C + (a[:, k:k + 1] * b[k:k + 1, :]).astype(np.float16)).astype(np.float16)
+    C = C.astype(np.float64)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    return np.maximum(C, 0.0) if relu else C
+
+
+def mutant_off_by_one_row(A, B, bias, relu):
+    C = _ref(A, B, bias, relu)
+    return np.roll(C, 1, axis=0) if C.shape[0] > 1 else C
+
+
+def mutant_f32_products(A, B, bias, relu):
+    C = (dec(A).astype(np.float32) @ dec(B).astype(np.float32)).astype(np.float64)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    return np.maximum(C, 0.0) if relu else C
+
+
+MUTANTS = [mutant_dropped_last_k, mutant_transposed_B, mutant_row_bias, mutant_bias_sign,
+           mutant_relu_before_bias, mutant_fp16_accumulator, mutant_off_by_one_row, mutant_f32_products]
+
+
+def test_reference_numpy_copy_passes_pins():
+    for pin in PINS:
+        pin(_ref)
+
+
+@pytest.mark.parametrize("mutant", MUTANTS, ids=lambda m: m.__name__)
+def test_planted_mistake_is_caught(mutant):
+    failed = []
+    for pin in PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"{mutant.__name__} passed every pin"
