@@ -1,0 +1,416 @@
+"""Benchmark of the fp16 GEMM (+bias+ReLU) path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one call of the GEMM entry point on one synthetic, HBM-resident
+problem of the chosen workload (default: M = N = K = 4096 with the fused
+bias+ReLU epilogue and fp16 output).  The L2 cache (126 MB) is flushed by
+writing a 256 MiB buffer before every step, outside the timed kernel.
+
+Timing: CUDA events on the launching stream around each step's launch, W
+untimed warm-up steps, K timed steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides, max over ranks.  `value` is the whole
+job's TFLOP/s = (2 M N K x K steps x ranks) / max-over-ranks GEMM time.
+
+With --gpus N > 1 (launched by torchrun) every rank solves its own problem of
+the same size: the problems are independent, there is no collective on the
+data path ("scaling": "weak").
+
+--impl reference times the CPU oracle (fp64 triple loop, OpenMP over rows) on
+a bounded row sample of the same workload, on the host cores; rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import tlg_workloads as wl  # noqa: E402
+
+METRIC = "TFLOP/s (fp16 GEMM, fp32 acc; +bias+ReLU) and % of B200 dense FP16 peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "gemm_bias_relu_4096_f16"
+DATASHEET_FP16_TFLOPS = 2250.0  # dense fp16 tensor peak, NVIDIA B200 datasheet
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tiled_dense_gemm_tlg_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch recorded from an ncu capture of the current kernel sources, else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def nvsmi_id(dev) -> str:
+    """nvidia-smi -i argument for a torch device (its UUID, independent of CUDA_VISIBLE_DEVICES)."""
+    import torch
+
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self._thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._thread:
+            self._thread.join(timeout=2)
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def cpu_oracle_rate(w: wl.Workload, target_s: float, threads: int, A=None, B=None, bias=None):
+    """Time the oracle on a row sample of the workload sized for about target_s seconds.
+    Returns (TFLOP/s, rows timed, seconds)."""
+    import oracle
+
+    if A is None:
+        A, B, bias = wl.workload_operands(w)
+    probe = max(1, min(w.M, 8))
+    t0 = time.perf_counter()
+    oracle.gemm(A[:probe], B, bias=bias, relu=w.bias_relu, threads=threads)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    rows = int(min(w.M, max(threads, probe * target_s / dt)))
+    rows = max(1, (rows // threads) * threads) if rows >= threads else rows
+    t0 = time.perf_counter()
+    oracle.gemm(A[:rows], B, bias=bias, relu=w.bias_relu, threads=threads)
+    dt = time.perf_counter() - t0
+    return 2.0 * rows * w.N * w.K / dt / 1e12, rows, dt
+
+
+def run_reference(args, w: wl.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+
+    threads = oracle.default_threads()
+    A, B, bias = wl.workload_operands(w)
+    # each step: a row sample sized so that warmup + steps stay within a few minutes
+    per_step = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    _, rows, _ = cpu_oracle_rate(w, per_step, threads, A, B, bias)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.gemm(A[:rows], B, bias=bias, relu=w.bias_relu, threads=threads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    flops = 2.0 * rows * w.N * w.K
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    sample = f"{rows} of {w.M} rows of the {w.name} workload per step (all N x K), fp64 oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: wl.Workload, kcfg):
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": w.out,
+            "epilogue": "bias_relu" if w.bias_relu else "none", "accumulate": "f32",
+            "inputs": "uniform[-1,1] fp16" if w.dist == "uniform" else "normal(0,1)*0.25 fp16",
+            "l2": f"flushed before every step ({FLUSH_BYTES >> 20} MiB write, untimed)",
+            "kernel_config": kcfg, "parallelism": "independent problem per GPU"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=wl.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="tlg", choices=["tlg", "reference"])
+    ap.add_argument("--config", default=None, help="JSON tlg_config override (tuning sweeps)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+
+    world, rank, local = dist_setup(args.gpus)
+    import tiled_dense_gemm_tlg_b200 as tlg
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    A, B, bias = wl.workload_operands(w, seed=rank)
+    dA, dB = A.to(dev), B.to(dev)
+    dbias = bias.to(dev) if bias is not None else None
+    dC = torch.empty((w.M, w.N), dtype=torch.float32 if w.out == "f32" else torch.float16, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    override = json.loads(args.config) if args.config else None
+    kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu)
+    if override:
+        kcfg.update(override)
+
+    def step():
+        if override:
+            tlg.tlg_gemm_ex(dA, dB, dbias, dC, out=w.out, config=override, stream=stream)
+        elif w.bias_relu:
+            tlg.tlg_gemm_bias_relu_f16(dA, dB, dbias, dC, stream=stream)
+        elif w.out == "f16":
+            tlg.tlg_gemm_f16f16(dA, dB, dC, stream=stream)
+        else:
+            tlg.tlg_gemm_f16f32(dA, dB, dC, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    rc, code = tlg.tlg_device_error(clear=True)
+    if rc != 0:
+        raise SystemExit(f"device error word {code:#x} during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(nvsmi_id(dev))
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(float(i))  # untimed: evicts A, B and C from L2
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    gemm_ms = sum(per_step_ms)
+    rc, code = tlg.tlg_device_error(clear=True)
+    if rc != 0:
+        raise SystemExit(f"device error word {code:#x} during the timed steps")
+
+    max_ms = max_over_ranks(gemm_ms, world)
+    total_flops = w.flops * args.steps * world
+    value = total_flops / (max_ms * 1e-3) / 1e12
+    ms_per_step = max_ms / args.steps
+
+    # ---- end to end through the public API: pinned host inputs -> device -> GEMM -> pinned host output
+    e2e = None
+    if not args.no_e2e:
+        hA, hB = A.pin_memory(), B.pin_memory()
+        hbias = bias.pin_memory() if bias is not None else None
+        hC = torch.empty(dC.shape, dtype=dC.dtype).pin_memory()
+        h2d = hA.numel() * 2 + hB.numel() * 2 + (hbias.numel() * 2 if hbias is not None else 0)
+        d2h = hC.numel() * hC.element_size()
+
+        def e2e_step():
+            dA.copy_(hA, non_blocking=True)
+            dB.copy_(hB, non_blocking=True)
+            if hbias is not None:
+                dbias.copy_(hbias, non_blocking=True)
+            step()
+            hC.copy_(dC, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))  # fp16 = bf16 rate (same nominal)
+    achieved = w.flops / (statistics.mean(per_step_ms) * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                "frac": achieved / peak, "traffic": load_traffic(w.name),
+                "peak_source": f"{peak_src} cuBLAS-class bf16 burst x 1.0 (fp16/bf16 nominal ratio)",
+                "frac_of_datasheet_fp16": achieved / DATASHEET_FP16_TFLOPS,
+                "algorithmic_flops_per_launch": w.flops, "algorithmic_bytes_per_launch": w.algorithmic_bytes}
+    if clk:
+        roofline["frac_of_clock_peak"] = achieved / (148 * 8192 * clk["sm_mhz"] * 1e6 / 1e12)
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        import oracle
+
+        threads = oracle.default_threads()
+        rate, rows, secs = cpu_oracle_rate(w, 10.0, threads, A, B, bias)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{rows} of {w.M} output rows (all N={w.N} columns, K={w.K}) in {secs:.1f} s, fp64"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": workload_config(w, kcfg),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "per_step_ms": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
+                        "max": max(per_step_ms)},
+        "kernel_source_hash": kernel_source_hash(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,178 @@
+/*
+ * tlg.h -- C interface of libtlg, a B200 (sm_100a) fp16 GEMM library.
+ *
+ * The operation is the block-tiled GEMM of the TileLang pages:
+ *
+ *   C = A . B      A: M x K fp16, row-major (K contiguous), row stride lda
+ *                  B: K x N fp16, row-major (N contiguous), row stride ldb
+ *                  C: M x N, row-major, row stride ldc
+ *
+ * accumulated in fp32 ("tilelang operator-compilation walkthrough",
+ * lqnn.cn/news/222844, section 2.1: one fp32 accumulator tile per output block,
+ * filled over the K loop; section 4.2: fp16 in, fp32 accumulate, fp16 out;
+ * "TileLang Python DSL practice", codechina.net/.../126997, section 3.2: the
+ * same product written to an fp32 C).  The fused variant applies a per-column
+ * bias and a ReLU before the fp16 store ("domestic-GPU TileLang adoption",
+ * xdnf.cn/news/333523, section 4.2).
+ *
+ * Conventions shared by every entry point below:
+ *
+ *  - All matrix pointers are DEVICE pointers (cudaMalloc, a caching
+ *    allocator, or managed memory) on the current CUDA device.  A host pointer
+ *    is rejected with TLG_ERR_INVALID_ARG instead of silently producing an
+ *    empty result (the pitfall named in "tilelang operator-compilation
+ *    walkthrough" section 5.2).
+ *  - The caller owns every buffer.  C is overwritten (no accumulate-into).
+ *    C must not overlap A, B or the bias.
+ *  - The call is asynchronous: it enqueues work on `stream` (a cudaStream_t;
+ *    NULL means the legacy default stream) and returns.  Calls are
+ *    stream-ordered and may be issued from several host threads.
+ *  - The library allocates no device memory.
+ *  - Alignment (a rule of the TMA engine that loads the tiles): A, B, C and
+ *    the bias must be 16-byte aligned, and lda*2, ldb*2 and ldc*sizeof(out)
+ *    must be multiples of 16 bytes.  Otherwise TLG_ERR_ALIGNMENT.
+ *  - Sizes: 0 <= M, N, K <= 2^31 - 257, and ceil(M/128)*ceil(N/64) below 2^31
+ *    (larger sizes give TLG_ERR_UNSUPPORTED); lda >= K, ldb >= N, ldc >= N.
+ *    M == 0 or N == 0: nothing is written, TLG_OK.  K == 0: the empty sum is
+ *    0, so C = 0 (bias variant: C = fp16(max(bias[col], 0))).
+ *  - The return value is the only error channel; nothing throws or aborts.
+ *    Errors found before launch leave C untouched.  An error of the launch
+ *    itself is TLG_ERR_CUDA.  Errors the kernel detects on the device (a
+ *    pipeline wait that exceeded its time limit) are not visible to the
+ *    asynchronous call; read them with tlg_device_error().
+ *  - Requires an sm_100 device (B200); other devices give TLG_ERR_UNSUPPORTED.
+ */
+#ifndef TLG_H
+#define TLG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tlg_status {
+    TLG_OK = 0,
+    TLG_ERR_INVALID_ARG = 1, /* negative size, null/host pointer, ld too small, overlap */
+    TLG_ERR_ALIGNMENT = 2,   /* pointer or row stride breaks the 16-byte rule */
+    TLG_ERR_UNSUPPORTED = 3, /* not an sm_100 device, size beyond 2^31-1, bad config */
+    TLG_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+    TLG_ERR_TIMEOUT = 5      /* a kernel reported a pipeline wait past its time limit */
+} tlg_status;
+
+/*
+ * C (fp32) = A . B with fp32 accumulation.
+ * Page: "TileLang Python DSL practice" (codechina.net/.../126997) section 3.2
+ * (fp16 A/B, fp32 C, fp32 accumulation).
+ */
+tlg_status tlg_gemm_f16f32(int64_t M, int64_t N, int64_t K,
+                           const void *A, int64_t lda,
+                           const void *B, int64_t ldb,
+                           float *C, int64_t ldc,
+                           void *stream);
+
+/*
+ * C (fp16) = round_to_nearest_even(A . B), fp32 accumulation.
+ * Page: "tilelang operator-compilation walkthrough" (lqnn.cn/news/222844)
+ * sections 2.1 and 4.2 (fp16 in, fp32 accumulator, fp16 C).
+ */
+tlg_status tlg_gemm_f16f16(int64_t M, int64_t N, int64_t K,
+                           const void *A, int64_t lda,
+                           const void *B, int64_t ldb,
+                           void *C, int64_t ldc,
+                           void *stream);
+
+/*
+ * C (fp16) = round_to_nearest_even(max(A . B + bias[col], 0)), fp32
+ * accumulation; the bias (N fp16 values, device memory, 16-byte aligned) is
+ * added in fp32 to the fp32 accumulator before the ReLU.
+ * Page: "domestic-GPU TileLang adoption" (xdnf.cn/news/333523) section 4.2
+ * (bias looked up at the output column, added, then max with 0).
+ */
+tlg_status tlg_gemm_bias_relu_f16(int64_t M, int64_t N, int64_t K,
+                                  const void *A, int64_t lda,
+                                  const void *B, int64_t ldb,
+                                  const void *bias,
+                                  void *C, int64_t ldc,
+                                  void *stream);
+
+/* ---------------------------------------------------------------- extended */
+
+/* Output type / epilogue selectors for tlg_gemm_ex. */
+typedef enum tlg_out { TLG_OUT_F32 = 0, TLG_OUT_F16 = 1 } tlg_out;
+typedef enum tlg_epilogue { TLG_EPI_NONE = 0, TLG_EPI_BIAS_RELU = 1 } tlg_epilogue;
+
+/*
+ * Kernel configuration.  Zero in any field means "choose for me" (the
+ * library's per-shape table, the analogue of the pages' cached tuned
+ * configurations: "tilelang operator-compilation walkthrough" section 5.3).
+ *   block_n     : output tile width per CTA, 64, 128 or 256 columns
+ *   stages      : depth of the shared-memory operand ring, 2..8
+ *   cta_group   : 1 (one SM per 128-row tile) or 2 (an SM pair per 256-row tile)
+ *   raster_group: number of tile rows walked together for L2 reuse, 1..64
+ *   max_ctas    : cap on resident CTAs (0 = one per SM)
+ * A combination the library does not provide gives TLG_ERR_UNSUPPORTED.
+ */
+typedef struct tlg_config {
+    int32_t block_n;
+    int32_t stages;
+    int32_t cta_group;
+    int32_t raster_group;
+    int32_t max_ctas;
+} tlg_config;
+
+/*
+ * The three entry points above in one call, with an explicit configuration
+ * (NULL = automatic).  bias must be NULL unless epilogue is
+ * TLG_EPI_BIAS_RELU, and the bias epilogue needs out == TLG_OUT_F16.
+ * Same arguments, ownership and errors as above.
+ */
+tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K,
+                       const void *A, int64_t lda,
+                       const void *B, int64_t ldb,
+                       const void *bias,
+                       void *C, int64_t ldc,
+                       tlg_out out, tlg_epilogue epilogue,
+                       const tlg_config *config,
+                       void *stream);
+
+/*
+ * The configuration the automatic choice would use for this shape, written
+ * to *config (never NULL).  Host-only; no CUDA call other than reading the
+ * current device's SM count.
+ */
+tlg_status tlg_choose_config(int64_t M, int64_t N, int64_t K, tlg_out out,
+                             tlg_epilogue epilogue, tlg_config *config);
+
+/*
+ * Device-side error report for the current device.  Synchronizes the device,
+ * reads the library's device error word and, if clear != 0, resets it.
+ * *code_out (may be NULL) receives the raw word: 0 when no kernel has
+ * reported an error; otherwise bit 0 = a pipeline wait ran past its limit,
+ * and one bit per role that gave up: bit 8 the TMA producer, bit 9 the MMA
+ * issuer, bit 10 the epilogue, bit 11 tlg_selftest_timeout.
+ * Returns TLG_ERR_TIMEOUT when the word is non-zero, TLG_ERR_CUDA when the
+ * synchronization fails, TLG_OK otherwise.
+ */
+tlg_status tlg_device_error(int clear, uint32_t *code_out);
+
+/*
+ * Self-test of the error path: launches one tiny kernel that waits on a
+ * pipeline barrier nothing will ever signal, with a limit of `limit_us`
+ * microseconds (1..1000000), on `stream`.  The wait gives up, the kernel
+ * records the timeout in the device error word and returns normally; no
+ * fault, trap or hang.  Read the result with tlg_device_error().
+ */
+tlg_status tlg_selftest_timeout(uint32_t limit_us, void *stream);
+
+/* Static string for a status code; never NULL. */
+const char *tlg_status_string(tlg_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t tlg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TLG_H */

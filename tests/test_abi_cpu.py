@@ -1,0 +1,88 @@
+"""CPU-side checks of the C ABI: the library builds and loads, exports every
+function include/tlg.h declares, and rejects bad arguments on the host before
+any CUDA call."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib_path():
+    from tiled_dense_gemm_tlg_b200 import build
+    return build.build()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "tlg.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tlg_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_three_entry_points():
+    names = header_functions()
+    for n in ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16"):
+        assert n in names
+
+
+def test_library_exports_every_declared_function(lib_path):
+    lib = ctypes.CDLL(lib_path)
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (tlg_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(header_functions()) <= exported
+
+
+def test_library_does_not_link_torch(lib_path):
+    out = subprocess.run(["ldd", lib_path], capture_output=True, text=True).stdout
+    assert "torch" not in out and "c10" not in out
+
+
+def test_binding_names_match_header(lib_path):
+    import tiled_dense_gemm_tlg_b200 as tlg
+    for name in header_functions():
+        assert hasattr(tlg, name), name
+    assert tlg.tlg_version() >= 100
+
+
+def test_status_strings(lib_path):
+    import tiled_dense_gemm_tlg_b200 as tlg
+    for s in range(6):
+        assert tlg.tlg_status_string(s).startswith("TLG_")
+    assert "unknown" in tlg.tlg_status_string(99)
+
+
+def test_host_side_rejections_need_no_gpu(lib_path):
+    import tiled_dense_gemm_tlg_b200 as tlg
+    lib = tlg.raw_library()
+    f = lib.tlg_gemm_f16f32
+    A = 1 << 20  # fake, 16-byte-aligned addresses: these checks never dereference them
+    assert f(-1, 8, 8, A, 8, A, 8, A, 8, None) == tlg.TLG_ERR_INVALID_ARG
+    assert f(8, 8, 8, None, 8, A, 8, A * 2, 8, None) == tlg.TLG_ERR_INVALID_ARG
+    assert f(8, 8, 8, A, 7, A, 8, A * 2, 8, None) == tlg.TLG_ERR_INVALID_ARG
+    assert f(8, 8, 8, A + 2, 8, A, 8, A * 2, 8, None) == tlg.TLG_ERR_ALIGNMENT
+    assert f(8, 8, 12, A, 12, A, 8, A * 2, 8, None) == tlg.TLG_ERR_ALIGNMENT
+    assert f(8, 8, 8, A, 8, A, 8, A + 64, 8, None) == tlg.TLG_ERR_INVALID_ARG  # C overlaps A
+    assert f(0, 8, 8, None, 8, None, 8, None, 8, None) == tlg.TLG_OK  # empty: nothing to do
+    assert lib.tlg_gemm_bias_relu_f16(8, 8, 8, A, 8, A, 8, None, A * 2, 8, None) == tlg.TLG_ERR_INVALID_ARG
+    assert lib.tlg_gemm_ex(8, 8, 8, A, 8, A, 8, A * 3, A * 2, 8, 0, 1, None, None) == tlg.TLG_ERR_UNSUPPORTED
+    assert lib.tlg_selftest_timeout(0, None) == tlg.TLG_ERR_INVALID_ARG
+
+
+def test_binding_validates_shapes(lib_path):
+    import torch
+
+    import tiled_dense_gemm_tlg_b200 as tlg
+    A = torch.zeros((4, 8), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        tlg.tlg_gemm_f16f32(A, torch.zeros((9, 8), dtype=torch.float16))
+    with pytest.raises(TypeError):
+        tlg.tlg_gemm_f16f32(A.float(), torch.zeros((8, 8), dtype=torch.float16))
+    with pytest.raises(ValueError):
+        tlg.tlg_gemm_f16f32(torch.zeros((8, 4), dtype=torch.float16).t(), torch.zeros((8, 8), dtype=torch.float16))

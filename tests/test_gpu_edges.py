@@ -1,0 +1,212 @@
+"""GPU edge cases through the C ABI: ragged shapes straddling every tile edge
+(with NaN-filled padding and guard bands that must stay untouched), every
+tile width the library builds, degenerate sizes, streams, argument errors and
+the bounded-wait error path."""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tlg_workloads as wl
+from gpu_util import Padded, gemm_padded
+
+pytestmark = pytest.mark.gpu
+
+SIZES = [1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 256, 257]
+OUTS = [("f32", False), ("f16", False), ("f16", True)]
+WIDTHS = [64, 128, 256]
+
+
+@pytest.fixture(scope="module")
+def tlg():
+    import tiled_dense_gemm_tlg_b200 as t
+    return t
+
+
+@pytest.fixture(scope="module")
+def lib(tlg):
+    return tlg.raw_library()
+
+
+def edge_cases():
+    cases = []
+    i = 0
+    for M in SIZES:
+        for N in (1, 17, 64, 129, 257):
+            for K in (1, 16, 63, 65, 129, 300):
+                out, br = OUTS[i % 3]
+                cases.append((M, N, K, out, br, WIDTHS[(i // 3) % 3]))
+                i += 1
+    return cases
+
+
+@pytest.mark.parametrize("M,N,K,out,bias_relu,block_n", edge_cases())
+def test_ragged_edges(lib, M, N, K, out, bias_relu, block_n):
+    A, B, bias = wl.make_operands(M, N, K, "uniform", bias=bias_relu, seed=M * 1000003 + N * 1009 + K)
+    got, guards = gemm_padded(lib, A, B, bias, out, config={"block_n": block_n}, extra=(8, 8, 4))
+    assert guards, "a write landed outside M x N, or padding was modified"
+    ref = oracle.gemm(A, B, bias=bias, relu=bias_relu, threads=4)
+    assert np.isfinite(got).all(), "NaN padding leaked into the product"
+    ok, worst, idx = oracle.within_tolerance(got, ref, out)
+    assert ok, f"worst err/bound {worst:.3g} at {idx}: got {got[idx]} ref {ref[idx]}"
+
+
+@pytest.mark.parametrize("block_n", WIDTHS)
+@pytest.mark.parametrize("out,bias_relu", OUTS)
+def test_every_width_on_multi_tile_ragged_shape(lib, block_n, out, bias_relu):
+    M, N, K = 700, 520, 1000  # several tiles each way, ragged in M, N and K, many k-blocks
+    A, B, bias = wl.make_operands(M, N, K, "normal025", bias=bias_relu, seed=5)
+    got, guards = gemm_padded(lib, A, B, bias, out, config={"block_n": block_n}, extra=(8, 16, 8))
+    assert guards
+    ref = oracle.gemm(A, B, bias=bias, relu=bias_relu)
+    ok, worst, idx = oracle.within_tolerance(got, ref, out)
+    assert ok, f"worst err/bound {worst:.3g} at {idx}"
+
+
+@pytest.mark.parametrize("raster_group,max_ctas", [(1, 0), (3, 0), (64, 0), (8, 1), (8, 7)])
+def test_scheduler_variants(lib, raster_group, max_ctas):
+    # fewer CTAs than tiles makes each CTA loop over many tiles and both TMEM accumulators
+    M, N, K = 1100, 900, 333
+    A, B, _ = wl.make_operands(M, N, K, "uniform", seed=6)
+    cfg = {"block_n": 128, "raster_group": raster_group, "max_ctas": max_ctas}
+    got, guards = gemm_padded(lib, A, B, None, "f32", config=cfg)
+    assert guards
+    ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B), "f32")
+    assert ok, f"worst err/bound {worst:.3g} at {idx}"
+
+
+def test_transpose_identity_on_gpu(tlg):
+    A, B, _ = wl.make_operands(304, 200, 136, "uniform", seed=8)  # every ld a multiple of 8
+    C1 = tlg.tlg_gemm_f16f32(A.cuda(), B.cuda())
+    C2 = tlg.tlg_gemm_f16f32(B.t().contiguous().cuda(), A.t().contiguous().cuda())
+    torch.cuda.synchronize()
+    assert torch.allclose(C1.t(), C2, atol=1e-2, rtol=2e-3)
+
+
+def test_identity_and_all_ones_exact(tlg):
+    B = wl.make_operands(1, 264, 264, "uniform", seed=9)[1]
+    I = torch.eye(264, dtype=torch.float16)
+    C = tlg.tlg_gemm_f16f32(I.cuda(), B.cuda())
+    assert torch.equal(C.cpu(), B.float())
+    C16 = tlg.tlg_gemm_f16f16(I.cuda(), B.cuda())
+    assert torch.equal(C16.cpu(), B)
+    ones = torch.ones((130, 1000), dtype=torch.float16)
+    C = tlg.tlg_gemm_f16f32(ones.cuda(), torch.ones((1000, 72), dtype=torch.float16).cuda())
+    assert (C == 1000.0).all()
+
+
+def test_bias_only_and_negative_bias(tlg):
+    M, N, K = 140, 136, 70
+    bias = (torch.rand(N) - 0.5).half()
+    Z = torch.zeros((M, K), dtype=torch.float16).cuda()
+    B = wl.make_operands(1, N, K, "uniform", seed=10)[1].cuda()
+    C = tlg.tlg_gemm_bias_relu_f16(Z, B, bias.cuda())
+    assert torch.equal(C.cpu(), torch.clamp(bias.float(), min=0).half().expand(M, N))
+    A = wl.make_operands(M, N, K, "uniform", seed=11)[0].cuda()
+    C = tlg.tlg_gemm_bias_relu_f16(A, B, torch.full((N,), -1000.0, dtype=torch.float16).cuda())
+    assert (C == 0).all()
+
+
+@pytest.mark.parametrize("out,bias_relu", OUTS)
+def test_k_zero_is_empty_sum(tlg, out, bias_relu):
+    M, N = 33, 40
+    A = torch.empty((M, 0), dtype=torch.float16, device="cuda")
+    B = torch.empty((0, N), dtype=torch.float16, device="cuda")
+    bias = (torch.rand(N) - 0.5).half().cuda()
+    if bias_relu:
+        C = tlg.tlg_gemm_bias_relu_f16(A, B, bias)
+        assert torch.equal(C, torch.clamp(bias.float(), min=0).half().expand(M, N))
+    else:
+        fn = tlg.tlg_gemm_f16f32 if out == "f32" else tlg.tlg_gemm_f16f16
+        C = fn(A, B, torch.full((M, N), float("nan"), dtype=torch.float32 if out == "f32" else torch.float16,
+                                device="cuda"))
+        assert (C == 0).all()
+
+
+def test_m_or_n_zero_writes_nothing(tlg):
+    A = torch.ones((0, 64), dtype=torch.float16, device="cuda")
+    B = torch.ones((64, 32), dtype=torch.float16, device="cuda")
+    assert tlg.tlg_gemm_f16f32(A, B).shape == (0, 32)
+    A = torch.ones((16, 64), dtype=torch.float16, device="cuda")
+    B = torch.ones((64, 0), dtype=torch.float16, device="cuda")
+    assert tlg.tlg_gemm_f16f16(A, B).shape == (16, 0)
+
+
+def test_runs_on_a_side_stream(tlg):
+    A, B, _ = wl.make_operands(520, 384, 256, "uniform", seed=12)
+    dA, dB = A.cuda(), B.cuda()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        C = torch.full((520, 384), float("nan"), device="cuda")
+        tlg.tlg_gemm_f16f32(dA, dB, C, stream=s)
+    s.synchronize()
+    ok, worst, _ = oracle.within_tolerance(C.double().cpu().numpy(), oracle.gemm(A, B), "f32")
+    assert ok, worst
+
+
+# --------------------------------------------------------------------------- argument errors
+
+def _call(lib, M, N, K, pa, lda, pb, ldb, pc, ldc):
+    return lib.tlg_gemm_f16f32(M, N, K, pa, lda, pb, ldb, pc, ldc, None)
+
+
+def test_host_pointer_is_rejected(tlg, lib):
+    A = torch.ones((64, 64), dtype=torch.float16)
+    B = torch.ones((64, 64), dtype=torch.float16)
+    C = torch.zeros((64, 64), dtype=torch.float32)
+    assert _call(lib, 64, 64, 64, A.data_ptr(), 64, B.data_ptr(), 64, C.data_ptr(), 64) == tlg.TLG_ERR_INVALID_ARG
+    dA, dB = A.cuda(), B.cuda()
+    assert _call(lib, 64, 64, 64, dA.data_ptr(), 64, dB.data_ptr(), 64, C.data_ptr(), 64) == tlg.TLG_ERR_INVALID_ARG
+    pinned = torch.zeros((64, 64), dtype=torch.float32).pin_memory()
+    assert _call(lib, 64, 64, 64, dA.data_ptr(), 64, dB.data_ptr(), 64, pinned.data_ptr(), 64) == tlg.TLG_ERR_INVALID_ARG
+    with pytest.raises(tlg.TlgError):
+        tlg.tlg_gemm_f16f32(A, B)  # the pitfall: CPU tensors must fail loudly, never return an empty result
+
+
+def test_argument_errors(tlg, lib):
+    A = torch.ones((64, 64), dtype=torch.float16, device="cuda")
+    B = torch.ones((64, 64), dtype=torch.float16, device="cuda")
+    C = torch.zeros((64, 64), dtype=torch.float32, device="cuda")
+    pa, pb, pc = A.data_ptr(), B.data_ptr(), C.data_ptr()
+    E = tlg
+    assert _call(lib, -1, 64, 64, pa, 64, pb, 64, pc, 64) == E.TLG_ERR_INVALID_ARG
+    assert _call(lib, 64, 64, 64, None, 64, pb, 64, pc, 64) == E.TLG_ERR_INVALID_ARG
+    assert _call(lib, 64, 64, 64, pa, 63, pb, 64, pc, 64) == E.TLG_ERR_INVALID_ARG
+    assert _call(lib, 64, 64, 64, pa, 64, pb, 64, pc, 60) == E.TLG_ERR_INVALID_ARG
+    assert _call(lib, 64, 64, 60, pa, 60 + 2, pb, 64, pc, 64) == E.TLG_ERR_ALIGNMENT
+    assert _call(lib, 64, 64, 64, pa + 2, 64, pb, 64, pc, 64) == E.TLG_ERR_ALIGNMENT
+    assert _call(lib, 64, 64, 64, pa, 64, pb, 64, pc + 4, 64) == E.TLG_ERR_ALIGNMENT
+    assert _call(lib, 2 ** 31, 64, 64, pa, 64, pb, 64, pc, 64) == E.TLG_ERR_UNSUPPORTED
+    # C overlapping an operand
+    big = torch.zeros((256, 64), dtype=torch.float32, device="cuda")
+    assert _call(lib, 64, 64, 64, big.data_ptr(), 64, pb, 64, big.data_ptr() + 1024, 64) == E.TLG_ERR_INVALID_ARG
+    assert _call(lib, 64, 64, 64, pa, 64, pb, 64, pc, 64) == E.TLG_OK
+    with pytest.raises(E.TlgError):
+        E.tlg_gemm_ex(A, B, config={"block_n": 96})
+    with pytest.raises(E.TlgError):
+        E.tlg_gemm_ex(A, B, config={"cta_group": 3})
+    torch.cuda.synchronize()
+
+
+def test_choose_config_matches_table(tlg):
+    for name, w in wl.WORKLOADS.items():
+        c = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu)
+        assert c["block_n"] in (64, 128, 256) and c["stages"] >= 2
+
+
+def test_timeout_path_reports_and_recovers(tlg):
+    rc, _ = tlg.tlg_device_error(clear=True)
+    assert rc == 0
+    tlg.tlg_selftest_timeout(2000)  # a wait nothing will satisfy, limited to 2 ms
+    rc, code = tlg.tlg_device_error(clear=True)
+    assert rc == tlg.TLG_ERR_TIMEOUT and (code & 1) and (code & (1 << 11)), hex(code)
+    rc, code = tlg.tlg_device_error(clear=True)
+    assert rc == 0 and code == 0
+    # the context is still usable afterwards
+    A, B, _ = wl.make_operands(130, 130, 130, "uniform", seed=13)
+    C = tlg.tlg_gemm_f16f32(A.cuda(), B.cuda())
+    ok, _, _ = oracle.within_tolerance(C.double().cpu().numpy(), oracle.gemm(A, B), "f32")
+    assert ok

@@ -1,0 +1,204 @@
+"""Python binding of libtlg, the B200 (sm_100a) fp16 GEMM library.
+
+Argument marshalling only: every step of the GEMM runs in the CUDA kernels of
+``libtlg.so`` behind the C interface in ``include/tlg.h``.  PyTorch supplies
+device memory and the current stream.  There is no CPU fallback: importing
+this package fails when the library has not been built, and a call with CPU
+tensors is rejected by the library (TLG_ERR_INVALID_ARG) rather than returning
+an empty result.
+
+Functions (same names as the C entry points):
+
+* ``tlg_gemm_f16f32(A, B, C=None)``        C fp32 = A.B
+* ``tlg_gemm_f16f16(A, B, C=None)``        C fp16 = A.B
+* ``tlg_gemm_bias_relu_f16(A, B, bias, C=None)``  C fp16 = max(A.B + bias, 0)
+* ``tlg_gemm_ex(...)``                     any of the above with an explicit configuration
+* ``tlg_choose_config``, ``tlg_device_error``, ``tlg_selftest_timeout``,
+  ``tlg_status_string``, ``tlg_version``
+
+A and B are 2-D fp16 tensors with unit stride along their last dimension
+(row-major); their row strides become lda / ldb.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtlg.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libtlg.so not found at {LIB_PATH}: build it with `python -m tiled_dense_gemm_tlg_b200.build` "
+        "(there is no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+TLG_OK, TLG_ERR_INVALID_ARG, TLG_ERR_ALIGNMENT, TLG_ERR_UNSUPPORTED, TLG_ERR_CUDA, TLG_ERR_TIMEOUT = range(6)
+TLG_OUT_F32, TLG_OUT_F16 = 0, 1
+TLG_EPI_NONE, TLG_EPI_BIAS_RELU = 0, 1
+
+EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
+            "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
+            "tlg_version")
+
+
+class tlg_config(ctypes.Structure):
+    _fields_ = [("block_n", ctypes.c_int32), ("stages", ctypes.c_int32), ("cta_group", ctypes.c_int32),
+                ("raster_group", ctypes.c_int32), ("max_ctas", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+_i64, _p, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+_lib.tlg_gemm_f16f32.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p]
+_lib.tlg_gemm_f16f16.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p]
+_lib.tlg_gemm_bias_relu_f16.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _p]
+_lib.tlg_gemm_ex.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i32, _i32,
+                             ctypes.POINTER(tlg_config), _p]
+_lib.tlg_choose_config.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config)]
+_lib.tlg_device_error.argtypes = [_i32, ctypes.POINTER(ctypes.c_uint32)]
+_lib.tlg_selftest_timeout.argtypes = [ctypes.c_uint32, _p]
+_lib.tlg_status_string.argtypes = [_i32]
+_lib.tlg_status_string.restype = ctypes.c_char_p
+_lib.tlg_version.restype = ctypes.c_int32
+for _name in ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
+              "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
+    getattr(_lib, _name).restype = _i32
+
+
+class TlgError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {tlg_status_string(status)}")
+
+
+def tlg_status_string(status: int) -> str:
+    return _lib.tlg_status_string(int(status)).decode()
+
+
+def tlg_version() -> int:
+    return int(_lib.tlg_version())
+
+
+def _check(rc: int, where: str):
+    if rc != TLG_OK:
+        raise TlgError(rc, where)
+
+
+def _stream_handle(stream, *tensors) -> int:
+    if stream is not None:
+        return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            return int(torch.cuda.current_stream(t.device).cuda_stream)
+    return 0
+
+
+def _mat(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or t.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D tensor")
+    if t.size(1) > 1 and t.stride(1) != 1:
+        raise ValueError(f"{name} must be row-major (unit stride along its last dimension)")
+    return t.data_ptr(), max(t.stride(0), t.size(1))
+
+
+def _shapes(A, B):
+    if A.dtype != torch.float16 or B.dtype != torch.float16:
+        raise TypeError("A and B must be fp16")
+    M, K = A.shape
+    K2, N = B.shape
+    if K != K2:
+        raise ValueError(f"inner dimensions differ: A is {tuple(A.shape)}, B is {tuple(B.shape)}")
+    return M, N, K
+
+
+def _out(C, M, N, dtype, like):
+    if C is None:
+        return torch.empty((M, N), dtype=dtype, device=like.device)
+    if C.dtype != dtype or tuple(C.shape) != (M, N):
+        raise ValueError(f"C must be {dtype} of shape ({M}, {N})")
+    return C
+
+
+def tlg_gemm_f16f32(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor | None = None, stream=None):
+    M, N, K = _shapes(A, B)
+    C = _out(C, M, N, torch.float32, A)
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    pc, ldc = _mat(C, "C")
+    _check(_lib.tlg_gemm_f16f32(M, N, K, pa, lda, pb, ldb, pc, ldc, _stream_handle(stream, A, B, C)),
+           "tlg_gemm_f16f32")
+    return C
+
+
+def tlg_gemm_f16f16(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor | None = None, stream=None):
+    M, N, K = _shapes(A, B)
+    C = _out(C, M, N, torch.float16, A)
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    pc, ldc = _mat(C, "C")
+    _check(_lib.tlg_gemm_f16f16(M, N, K, pa, lda, pb, ldb, pc, ldc, _stream_handle(stream, A, B, C)),
+           "tlg_gemm_f16f16")
+    return C
+
+
+def tlg_gemm_bias_relu_f16(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor,
+                           C: torch.Tensor | None = None, stream=None):
+    M, N, K = _shapes(A, B)
+    if bias.dtype != torch.float16 or bias.dim() != 1 or bias.numel() != N or (N > 1 and bias.stride(0) != 1):
+        raise ValueError(f"bias must be a contiguous fp16 vector of length {N}")
+    C = _out(C, M, N, torch.float16, A)
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    pc, ldc = _mat(C, "C")
+    _check(_lib.tlg_gemm_bias_relu_f16(M, N, K, pa, lda, pb, ldb, bias.data_ptr(), pc, ldc,
+                                       _stream_handle(stream, A, B, C)), "tlg_gemm_bias_relu_f16")
+    return C
+
+
+def tlg_gemm_ex(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None = None,
+                C: torch.Tensor | None = None, out: str = "f32", config: dict | None = None, stream=None):
+    """Explicit-configuration form; ``out`` is "f32" or "f16"; a bias selects the bias+ReLU epilogue."""
+    M, N, K = _shapes(A, B)
+    o = TLG_OUT_F32 if out == "f32" else TLG_OUT_F16
+    C = _out(C, M, N, torch.float32 if o == TLG_OUT_F32 else torch.float16, A)
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    pc, ldc = _mat(C, "C")
+    cfg = None
+    if config is not None:
+        cfg = tlg_config(**{k: int(v) for k, v in config.items()})
+    epi = TLG_EPI_BIAS_RELU if bias is not None else TLG_EPI_NONE
+    _check(_lib.tlg_gemm_ex(M, N, K, pa, lda, pb, ldb, bias.data_ptr() if bias is not None else None,
+                            pc, ldc, o, epi, ctypes.byref(cfg) if cfg is not None else None,
+                            _stream_handle(stream, A, B, C)), "tlg_gemm_ex")
+    return C
+
+
+def tlg_choose_config(M: int, N: int, K: int, out: str = "f32", bias_relu: bool = False) -> dict:
+    cfg = tlg_config()
+    _check(_lib.tlg_choose_config(M, N, K, TLG_OUT_F32 if out == "f32" else TLG_OUT_F16,
+                                  TLG_EPI_BIAS_RELU if bias_relu else TLG_EPI_NONE, ctypes.byref(cfg)),
+           "tlg_choose_config")
+    return cfg.as_dict()
+
+
+def tlg_device_error(clear: bool = True):
+    """(status, raw word) of the device error word of the current device; synchronizes."""
+    code = ctypes.c_uint32(0)
+    rc = _lib.tlg_device_error(int(bool(clear)), ctypes.byref(code))
+    return rc, int(code.value)
+
+
+def tlg_selftest_timeout(limit_us: int, stream=None):
+    _check(_lib.tlg_selftest_timeout(int(limit_us), _stream_handle(stream)), "tlg_selftest_timeout")
+
+
+def raw_library():
+    """The ctypes handle of libtlg.so, for callers that marshal their own pointers."""
+    return _lib
