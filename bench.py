@@ -205,11 +205,16 @@ def cpu_oracle_rate(w: wl.Workload, target_s: float, threads: int, A=None, B=Non
 
     if A is None:
         A, B, bias = wl.workload_operands(w)
-    probe = max(1, min(w.M, 8))
-    t0 = time.perf_counter()
-    oracle.gemm(A[:probe], B, bias=bias, relu=w.bias_relu, threads=threads)
-    dt = max(time.perf_counter() - t0, 1e-6)
-    rows = int(min(w.M, max(threads, probe * target_s / dt)))
+    # grow a row sample until it takes a tenth of the target, then scale to the target
+    probe = max(1, min(w.M, threads))
+    while True:
+        t0 = time.perf_counter()
+        oracle.gemm(A[:probe], B, bias=bias, relu=w.bias_relu, threads=threads)
+        dt = max(time.perf_counter() - t0, 1e-6)
+        if dt >= target_s / 10 or probe >= w.M:
+            break
+        probe = min(w.M, probe * 4)
+    rows = int(min(w.M, max(probe, probe * target_s / dt)))
     rows = max(1, (rows // threads) * threads) if rows >= threads else rows
     t0 = time.perf_counter()
     oracle.gemm(A[:rows], B, bias=bias, relu=w.bias_relu, threads=threads)
@@ -288,9 +293,7 @@ def main(argv=None):
     dC = torch.empty((w.M, w.N), dtype=torch.float32 if w.out == "f32" else torch.float16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     override = json.loads(args.config) if args.config else None
-    kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu)
-    if override:
-        kcfg.update(override)
+    kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu, request=override)
 
     def step():
         if override:

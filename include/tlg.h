@@ -137,9 +137,12 @@ tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K,
                        void *stream);
 
 /*
- * The configuration the automatic choice would use for this shape, written
- * to *config (never NULL).  Host-only; no CUDA call other than reading the
- * current device's SM count.
+ * Resolve a configuration for this shape.  On input *config (never NULL)
+ * holds the requested fields, zero meaning "choose for me" (all zero: the
+ * automatic choice); on output it holds the configuration tlg_gemm_ex would
+ * run, every field filled in.  TLG_ERR_UNSUPPORTED if the request names a
+ * combination the library does not provide.  No kernel is launched; the only
+ * CUDA calls read the current device's attributes.
  */
 tlg_status tlg_choose_config(int64_t M, int64_t N, int64_t K, tlg_out out,
                              tlg_epilogue epilogue, tlg_config *config);

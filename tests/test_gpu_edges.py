@@ -18,6 +18,8 @@ pytestmark = pytest.mark.gpu
 SIZES = [1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 256, 257]
 OUTS = [("f32", False), ("f16", False), ("f16", True)]
 WIDTHS = [64, 128, 256]
+# every tile shape the library builds: (CTAs per tile, tile width)
+TILES = [(1, 64), (1, 128), (1, 256), (2, 128), (2, 256)]
 
 
 @pytest.fixture(scope="module")
@@ -38,15 +40,16 @@ def edge_cases():
         for N in (1, 17, 64, 129, 257):
             for K in (1, 16, 63, 65, 129, 300):
                 out, br = OUTS[i % 3]
-                cases.append((M, N, K, out, br, WIDTHS[(i // 3) % 3]))
+                cases.append((M, N, K, out, br, TILES[(i // 3) % len(TILES)]))
                 i += 1
     return cases
 
 
-@pytest.mark.parametrize("M,N,K,out,bias_relu,block_n", edge_cases())
-def test_ragged_edges(lib, M, N, K, out, bias_relu, block_n):
+@pytest.mark.parametrize("M,N,K,out,bias_relu,tile", edge_cases())
+def test_ragged_edges(lib, M, N, K, out, bias_relu, tile):
     A, B, bias = wl.make_operands(M, N, K, "uniform", bias=bias_relu, seed=M * 1000003 + N * 1009 + K)
-    got, guards = gemm_padded(lib, A, B, bias, out, config={"block_n": block_n}, extra=(8, 8, 4))
+    cfg = {"cta_group": tile[0], "block_n": tile[1]}
+    got, guards = gemm_padded(lib, A, B, bias, out, config=cfg, extra=(8, 8, 4))
     assert guards, "a write landed outside M x N, or padding was modified"
     ref = oracle.gemm(A, B, bias=bias, relu=bias_relu, threads=4)
     assert np.isfinite(got).all(), "NaN padding leaked into the product"
@@ -54,24 +57,26 @@ def test_ragged_edges(lib, M, N, K, out, bias_relu, block_n):
     assert ok, f"worst err/bound {worst:.3g} at {idx}: got {got[idx]} ref {ref[idx]}"
 
 
-@pytest.mark.parametrize("block_n", WIDTHS)
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("out,bias_relu", OUTS)
-def test_every_width_on_multi_tile_ragged_shape(lib, block_n, out, bias_relu):
+def test_every_tile_on_multi_tile_ragged_shape(lib, tile, out, bias_relu):
     M, N, K = 700, 520, 1000  # several tiles each way, ragged in M, N and K, many k-blocks
     A, B, bias = wl.make_operands(M, N, K, "normal025", bias=bias_relu, seed=5)
-    got, guards = gemm_padded(lib, A, B, bias, out, config={"block_n": block_n}, extra=(8, 16, 8))
+    cfg = {"cta_group": tile[0], "block_n": tile[1]}
+    got, guards = gemm_padded(lib, A, B, bias, out, config=cfg, extra=(8, 16, 8))
     assert guards
     ref = oracle.gemm(A, B, bias=bias, relu=bias_relu)
     ok, worst, idx = oracle.within_tolerance(got, ref, out)
     assert ok, f"worst err/bound {worst:.3g} at {idx}"
 
 
-@pytest.mark.parametrize("raster_group,max_ctas", [(1, 0), (3, 0), (64, 0), (8, 1), (8, 7)])
-def test_scheduler_variants(lib, raster_group, max_ctas):
+@pytest.mark.parametrize("tile", [(1, 128), (2, 256)])
+@pytest.mark.parametrize("raster_group,max_ctas", [(1, 0), (3, 0), (64, 0), (8, 2), (8, 7)])
+def test_scheduler_variants(lib, tile, raster_group, max_ctas):
     # fewer CTAs than tiles makes each CTA loop over many tiles and both TMEM accumulators
     M, N, K = 1100, 900, 333
     A, B, _ = wl.make_operands(M, N, K, "uniform", seed=6)
-    cfg = {"block_n": 128, "raster_group": raster_group, "max_ctas": max_ctas}
+    cfg = {"cta_group": tile[0], "block_n": tile[1], "raster_group": raster_group, "max_ctas": max_ctas}
     got, guards = gemm_padded(lib, A, B, None, "f32", config=cfg)
     assert guards
     ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B), "f32")
@@ -99,7 +104,7 @@ def test_identity_and_all_ones_exact(tlg):
 
 
 def test_bias_only_and_negative_bias(tlg):
-    M, N, K = 140, 136, 70
+    M, N, K = 140, 136, 72
     bias = (torch.rand(N) - 0.5).half()
     Z = torch.zeros((M, K), dtype=torch.float16).cuda()
     B = wl.make_operands(1, N, K, "uniform", seed=10)[1].cuda()
@@ -188,6 +193,8 @@ def test_argument_errors(tlg, lib):
         E.tlg_gemm_ex(A, B, config={"block_n": 96})
     with pytest.raises(E.TlgError):
         E.tlg_gemm_ex(A, B, config={"cta_group": 3})
+    with pytest.raises(E.TlgError):
+        E.tlg_gemm_ex(A, B, config={"cta_group": 2, "block_n": 64})
     torch.cuda.synchronize()
 
 
@@ -206,7 +213,7 @@ def test_timeout_path_reports_and_recovers(tlg):
     rc, code = tlg.tlg_device_error(clear=True)
     assert rc == 0 and code == 0
     # the context is still usable afterwards
-    A, B, _ = wl.make_operands(130, 130, 130, "uniform", seed=13)
+    A, B, _ = wl.make_operands(130, 136, 136, "uniform", seed=13)
     C = tlg.tlg_gemm_f16f32(A.cuda(), B.cuda())
     ok, _, _ = oracle.within_tolerance(C.double().cpu().numpy(), oracle.gemm(A, B), "f32")
     assert ok

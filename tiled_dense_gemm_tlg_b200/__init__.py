@@ -180,8 +180,10 @@ def tlg_gemm_ex(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None = No
     return C
 
 
-def tlg_choose_config(M: int, N: int, K: int, out: str = "f32", bias_relu: bool = False) -> dict:
-    cfg = tlg_config()
+def tlg_choose_config(M: int, N: int, K: int, out: str = "f32", bias_relu: bool = False,
+                      request: dict | None = None) -> dict:
+    """The configuration tlg_gemm_ex would run for this shape (request fields of 0 = automatic)."""
+    cfg = tlg_config(**{k: int(v) for k, v in (request or {}).items()})
     _check(_lib.tlg_choose_config(M, N, K, TLG_OUT_F32 if out == "f32" else TLG_OUT_F16,
                                   TLG_EPI_BIAS_RELU if bias_relu else TLG_EPI_NONE, ctypes.byref(cfg)),
            "tlg_choose_config")

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "tlg.h"
@@ -86,42 +87,49 @@ bool overlaps(uintptr_t a0, uintptr_t a1, uintptr_t b0, uintptr_t b1) { return a
 // --------------------------------------------------------------------------- configurations
 
 struct KernelCfg {
+  int cta_group;
   int block_n;
   int stages;
+  double eff;  // fraction of the MMA peak one tile sustains (used to rank tile shapes)
 };
 
-// The stage count each tile width is built with: as many operand slots as
-// fit next to each other in 227 KB of shared memory (48 KB, 32 KB, 24 KB per
-// slot for block_n 256, 128, 64).
-constexpr KernelCfg kBuilt[] = {{256, 4}, {128, 6}, {64, 8}};
+// Tile shapes the library is built with.  A tile is 128*cta_group rows by
+// block_n columns; `stages` is the deepest operand ring that fits in 227 KB of
+// shared memory next to the barriers.  Per-CTA ring slot: 16 KB of A plus
+// 128*block_n/cta_group bytes of B.
+// `eff` is measured: TFLOP/s of each shape on a B200 at M = N = K = 4096 and
+// 8192 after dividing out the wave count, relative to the 2 x 256 pair tile.
+constexpr KernelCfg kBuilt[] = {
+    {1, 64, 8, 0.35}, {1, 128, 6, 0.60}, {1, 256, 4, 0.90}, {2, 128, 8, 0.60}, {2, 256, 6, 1.00}};
 
-int built_stages(int block_n) {
+const KernelCfg *find_built(int cta_group, int block_n) {
   for (const KernelCfg &k : kBuilt)
-    if (k.block_n == block_n) return k.stages;
-  return 0;
+    if (k.cta_group == cta_group && k.block_n == block_n) return &k;
+  return nullptr;
 }
 
-// Pick the tile width: fewest estimated SM-time units, counting whole waves of
-// tiles over the SMs and a per-tile efficiency that drops for narrow tiles
-// (the 128 x N x 16 MMA reads all of A for every N, so shared-memory bandwidth
-// binds below N = 128).
+// Pick the tile shape with the fewest estimated SM-time units: whole waves of
+// tiles over the available CTAs (pairs), times the tile's work over its
+// sustained fraction of the MMA peak.  Narrow and single-SM tiles sustain less
+// because each 128-row MMA reads all of its A tile from shared memory for
+// every block_n columns it produces.
 void choose(int64_t M, int64_t N, int sms, tlg_config *c) {
-  const int widths[] = {256, 128, 64};
-  const double eff[] = {1.0, 0.95, 0.70};
   double best = 0;
-  int best_n = 256;
-  for (int i = 0; i < 3; ++i) {
-    const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + widths[i] - 1) / widths[i]);
-    const int64_t waves = (tiles + sms - 1) / sms;
-    const double cost = static_cast<double>(waves) * widths[i] / eff[i];
-    if (i == 0 || cost < best) {
+  const KernelCfg *pick = &kBuilt[0];
+  for (const KernelCfg &k : kBuilt) {
+    const int64_t tile_m = 128 * k.cta_group;
+    const int64_t tiles = ((M + tile_m - 1) / tile_m) * ((N + k.block_n - 1) / k.block_n);
+    const int64_t units = sms / k.cta_group;
+    const int64_t waves = (tiles + units - 1) / units;
+    const double cost = static_cast<double>(waves) * tile_m * k.block_n / (k.cta_group * k.eff);
+    if (&k == &kBuilt[0] || cost < best * 0.999) {
       best = cost;
-      best_n = widths[i];
+      pick = &k;
     }
   }
-  c->block_n = best_n;
-  c->stages = built_stages(best_n);
-  c->cta_group = 1;
+  c->block_n = pick->block_n;
+  c->stages = pick->stages;
+  c->cta_group = pick->cta_group;
   c->raster_group = 8;
   c->max_ctas = 0;
 }
@@ -129,15 +137,21 @@ void choose(int64_t M, int64_t N, int sms, tlg_config *c) {
 tlg_status resolve_config(int64_t M, int64_t N, int sms, const tlg_config *req, tlg_config *out) {
   choose(M, N, sms, out);
   if (req == nullptr) return TLG_OK;
-  if (req->block_n != 0) {
-    if (built_stages(req->block_n) == 0) return TLG_ERR_UNSUPPORTED;
-    out->block_n = req->block_n;
-    out->stages = built_stages(req->block_n);
+  int cg = req->cta_group != 0 ? req->cta_group : out->cta_group;
+  int bn = req->block_n != 0 ? req->block_n : out->block_n;
+  const KernelCfg *k = find_built(cg, bn);
+  if (k == nullptr) {
+    // a width given alone may exist only for the other CTA-group size
+    if (req->cta_group == 0 && req->block_n != 0) {
+      cg = 3 - cg;
+      k = find_built(cg, bn);
+    }
+    if (k == nullptr) return TLG_ERR_UNSUPPORTED;
   }
-  if (req->stages != 0) {
-    if (req->stages != out->stages) return TLG_ERR_UNSUPPORTED;
-  }
-  if (req->cta_group != 0 && req->cta_group != 1) return TLG_ERR_UNSUPPORTED;
+  out->cta_group = cg;
+  out->block_n = bn;
+  out->stages = k->stages;
+  if (req->stages != 0 && req->stages != k->stages) return TLG_ERR_UNSUPPORTED;
   if (req->raster_group != 0) {
     if (req->raster_group < 1 || req->raster_group > 64) return TLG_ERR_UNSUPPORTED;
     out->raster_group = req->raster_group;
@@ -162,28 +176,58 @@ bool encode_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
-tlg_status launch_gemm(int dev, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                       const GemmParams &p, int grid, cudaStream_t stream) {
-  using Plan = SmemPlan<BN, STAGES>;
-  auto kernel = gemm_sm100_kernel<BN, STAGES, OUT_F16, BIAS_RELU>;
-  static bool attr_set[kMaxDevices] = {};
+struct LaunchState {
+  bool attr_set = false;
+  int max_clusters = 0;  // co-resident clusters of this kernel (cta_group 2)
+};
+
+// Launch one kernel instantiation: persistent grid of one CTA per SM (or one
+// cluster per SM pair, limited to the clusters that fit at once), capped by
+// the tile count and max_ctas.
+template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
+tlg_status launch_gemm(int dev, int sms, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                       const GemmParams &p, int64_t tiles, int max_ctas, cudaStream_t stream) {
+  using Plan = SmemPlan<CG, BN, STAGES>;
+  auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU>;
+  static LaunchState state[kMaxDevices];
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Plan::kDynamicBytes;
+  cfg.stream = stream;
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!attr_set[dev]) {
+    LaunchState &st = state[dev];
+    if (!st.attr_set) {
       if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Plan::kDynamicBytes) != cudaSuccess) {
         cudaGetLastError();
         return TLG_ERR_CUDA;
       }
-      attr_set[dev] = true;
+      if (CG == 2) {
+        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
+          cudaGetLastError();
+          return TLG_ERR_CUDA;
+        }
+        st.max_clusters = n;
+      }
+      st.attr_set = true;
     }
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Plan::kDynamicBytes;
-  cfg.stream = stream;
+  int64_t units = CG == 2 ? state[dev].max_clusters : sms;
+  if (max_ctas > 0) units = std::min<int64_t>(units, std::max(1, max_ctas / CG));
+  units = std::min<int64_t>(units, tiles);
+  cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, p);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -193,12 +237,22 @@ tlg_status launch_gemm(int dev, const CUtensorMap &tmA, const CUtensorMap &tmB,
 }
 
 template <bool OUT_F16, bool BIAS_RELU>
-tlg_status dispatch(int dev, const tlg_config &c, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                    const GemmParams &p, int grid, cudaStream_t s) {
+tlg_status dispatch(int dev, int sms, const tlg_config &c, const CUtensorMap &tmA,
+                    const CUtensorMap &tmB, const GemmParams &p, cudaStream_t s) {
+  const int64_t tile_m = 128 * c.cta_group;
+  const int64_t tiles = ((p.M + tile_m - 1) / tile_m) * ((p.N + c.block_n - 1) / c.block_n);
+  const int mc = c.max_ctas;
+  if (c.cta_group == 1) {
+    switch (c.block_n) {
+      case 256: return launch_gemm<1, 256, 4, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
+      case 128: return launch_gemm<1, 128, 6, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
+      case 64: return launch_gemm<1, 64, 8, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
+      default: return TLG_ERR_UNSUPPORTED;
+    }
+  }
   switch (c.block_n) {
-    case 256: return launch_gemm<256, 4, OUT_F16, BIAS_RELU>(dev, tmA, tmB, p, grid, s);
-    case 128: return launch_gemm<128, 6, OUT_F16, BIAS_RELU>(dev, tmA, tmB, p, grid, s);
-    case 64: return launch_gemm<64, 8, OUT_F16, BIAS_RELU>(dev, tmA, tmB, p, grid, s);
+    case 256: return launch_gemm<2, 256, 6, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
+    case 128: return launch_gemm<2, 128, 8, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
     default: return TLG_ERR_UNSUPPORTED;
   }
 }
@@ -291,14 +345,9 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
   p.K = int(K);
   p.raster_group = cfg.raster_group;
   p.limit_ns = kWaitLimitNs;
-  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + cfg.block_n - 1) / cfg.block_n);
-  int64_t grid = info.sm_count;
-  if (cfg.max_ctas > 0 && cfg.max_ctas < grid) grid = cfg.max_ctas;
-  if (tiles < grid) grid = tiles;
-
-  if (!f16) return dispatch<false, false>(dev, cfg, tmA, tmB, p, int(grid), s);
-  if (br) return dispatch<true, true>(dev, cfg, tmA, tmB, p, int(grid), s);
-  return dispatch<true, false>(dev, cfg, tmA, tmB, p, int(grid), s);
+  if (!f16) return dispatch<false, false>(dev, info.sm_count, cfg, tmA, tmB, p, s);
+  if (br) return dispatch<true, true>(dev, info.sm_count, cfg, tmA, tmB, p, s);
+  return dispatch<true, false>(dev, info.sm_count, cfg, tmA, tmB, p, s);
 }
 
 }  // namespace
@@ -333,7 +382,6 @@ tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K, const void *A, int64_t l
 
 tlg_status tlg_choose_config(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_epilogue epilogue,
                              tlg_config *config) {
-  (void)K;
   (void)out;
   (void)epilogue;
   if (config == nullptr || M < 0 || N < 0 || K < 0) return TLG_ERR_INVALID_ARG;
@@ -341,8 +389,8 @@ tlg_status tlg_choose_config(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_e
   DeviceInfo info;
   const tlg_status ds = current_device(&dev, &info);
   if (ds != TLG_OK) return ds;
-  choose(M, N, info.sm_count, config);
-  return TLG_OK;
+  const tlg_config req = *config;
+  return resolve_config(M, N, info.sm_count, &req, config);
 }
 
 tlg_status tlg_device_error(int clear, uint32_t *code_out) {

@@ -37,10 +37,14 @@ constexpr int kThreads = 192;
 
 __device__ uint32_t g_device_error;
 
-template <int BN, int STAGES>
+// Shared-memory plan of one CTA.  CG CTAs (1 or 2) compute one tile of
+// 128*CG rows by BN columns; each CTA stages its own 128 rows of A and its own
+// BN/CG columns of B per k-block.
+template <int CG, int BN, int STAGES>
 struct SmemPlan {
+  static constexpr int kBNc = BN / CG;  // B columns held by one CTA
   static constexpr uint32_t kABytes = kBM * kBK * 2;
-  static constexpr uint32_t kBBytes = kBK * BN * 2;
+  static constexpr uint32_t kBBytes = kBK * kBNc * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kBarOffset = STAGES * kStageBytes;
   static constexpr uint32_t kNumBars = 2 * STAGES + 4 + 1;  // full, empty, tmem full/empty x2, drain
@@ -48,6 +52,7 @@ struct SmemPlan {
   static constexpr uint32_t kBytes = kMiscOffset + 16;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack to align the base to 1024
   static constexpr uint32_t kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
+  static_assert(kBNc % 64 == 0, "each CTA's B slice must be whole 64-column swizzle blocks");
   static_assert(kTmemCols <= 512, "two accumulators must fit in TMEM");
   static_assert(kDynamicBytes <= 232448, "shared memory per CTA exceeded");
 };
@@ -132,12 +137,14 @@ __device__ __forceinline__ void store_chunk(const GemmParams &p, int row, int co
   }
 }
 
-template <int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
+template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
-  using Plan = SmemPlan<BN, STAGES>;
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128 or 256");
+  using Plan = SmemPlan<CG, BN, STAGES>;
+  constexpr int kTileM = kBM * CG;
+  static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -156,7 +163,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_m = (p.M + kBM - 1) / kBM;
+  // Work unit = one tile per CTA group: a CTA (CG == 1) or a cluster of two (CG == 2).
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+  const int unit = (CG == 2) ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int num_units = (CG == 2) ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+  const bool leader = rank == 0;
+  const int num_m = (p.M + kTileM - 1) / kTileM;
   const int num_n = (p.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (p.K + kBK - 1) / kBK;
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
+      mbar_init(tempty_bar(a), 4 * CG);  // one arrive per epilogue warp of each CTA
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
@@ -177,36 +189,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), Plan::kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<CG>(smem_u32(tmem_holder), Plan::kTmemCols);
+    tmem_relinquish<CG>();
   }
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (CG == 2)
+    cluster_sync_all();  // both CTAs' barriers exist before either signals the other
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_holder);
 
   if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- producer
+    // ---------------------------------------------------------------- producer (every CTA)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_parity = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+    for (int t = unit; t < num_tiles && ok; t += num_units) {
       int mb, nb;
       tile_coords(t, num_m, num_n, p.raster_group, mb, nb);
+      const int a_row = mb * kTileM + static_cast<int>(rank) * kBM;
+      const int b_col = nb * BN + static_cast<int>(rank) * Plan::kBNc;
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
                        &g_device_error)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(full_bar(stage), Plan::kStageBytes);
-        tma_load_2d(smem_u32(sA + stage * Plan::kABytes), &tmA, full_bar(stage), kb * kBK,
-                    mb * kBM);
+        const uint32_t a_dst = smem_u32(sA + stage * Plan::kABytes);
+        const uint32_t b_dst = smem_u32(sB + stage * Plan::kBBytes);
+        if constexpr (CG == 1) {
+          mbar_arrive_expect_tx(full_bar(stage), Plan::kStageBytes);
+          tma_load_2d(a_dst, &tmA, full_bar(stage), kb * kBK, a_row);
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c)
-          tma_load_2d(smem_u32(sB + stage * Plan::kBBytes + c * 8192), &tmB, full_bar(stage),
-                      nb * BN + c * 64, kb * kBK);
+          for (int c = 0; c < Plan::kBNc / 64; ++c)
+            tma_load_2d(b_dst + c * 8192, &tmB, full_bar(stage), b_col + c * 64, kb * kBK);
+        } else {
+          // The leader's full barrier counts the bytes of both CTAs' loads.
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * Plan::kStageBytes);
+          const uint32_t bar = mapa_shared(full_bar(stage), 0);
+          tma_load_2d_pair(a_dst, &tmA, bar, kb * kBK, a_row);
+#pragma unroll
+          for (int c = 0; c < Plan::kBNc / 64; ++c)
+            tma_load_2d_pair(b_dst + c * 8192, &tmB, bar, b_col + c * 64, kb * kBK);
+        }
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) {
@@ -216,8 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (ok) {
-      // Tail: wait until the MMA warp has released every slot, so that no
-      // commit-arrive is still on its way to this CTA's barriers at exit.
+      // Tail: wait until every slot has been released, so no commit-arrive is
+      // still on its way to this CTA's barriers when it exits.
       for (int i = 0; i < STAGES; ++i) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
                        &g_device_error)) {
@@ -230,22 +258,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (!ok) {
-      // Let every copy already issued land before the CTA's shared memory goes away.
+    if (!ok && leader) {
+      // Let the copies already issued land before shared memory goes away.
       for (int s = 0; s < STAGES; ++s)
         if (issued_mask & (1u << s))
           mbar_wait(full_bar(s), (issued_parity >> s) & 1u, nullptr, p.limit_ns, kRoleProducer,
                     &g_device_error);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = make_idesc_f16(kBM, BN);
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------------------------------------------------------- MMA issuer (leader CTA)
+    constexpr uint32_t idesc = make_idesc_f16(kTileM, BN);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+    for (int t = unit; t < num_tiles && ok; t += num_units) {
       if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
                      &g_device_error)) {
         ok = false;
@@ -266,38 +294,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(b0 + kk * 16 * 128, 8192, 1024);
-          mma_f16_ss(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
-        mma_commit(empty_bar(stage));
+        mma_commit<CG>(empty_bar(stage));
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      mma_commit(tfull_bar(acc));
+      mma_commit<CG>(tfull_bar(acc));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
     if (!ok) {
       // Wait for the MMAs already in flight before TMEM and shared memory are released.
-      mma_commit(drain_bar);
+      mma_commit_local<CG>(drain_bar);
       mbar_wait(drain_bar, 0, nullptr, p.limit_ns, kRoleMma, &g_device_error);
     }
   } else if (warp >= 2) {
-    // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- epilogue (every CTA)
     const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ...
-    const int row_in_tile = quarter * 32 + lane;
+    const int row_in_tile = static_cast<int>(rank) * kBM + quarter * 32 + lane;
+    const uint32_t release_bar0 = (CG == 2) ? mapa_shared(tempty_bar(0), 0) : tempty_bar(0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    for (int t = unit; t < num_tiles; t += num_units) {
       int mb, nb;
       tile_coords(t, num_m, num_n, p.raster_group, mb, nb);
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.limit_ns, kRoleEpilogue,
                      &g_device_error))
         break;
       tc_fence_after_sync();
-      const int row = mb * kBM + row_in_tile;
+      const int row = mb * kTileM + row_in_tile;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
@@ -309,18 +338,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row < p.M && col0 < p.N) store_chunk<OUT_F16, BIAS_RELU>(p, row, col0, r);
       }
       tc_fence_before_sync();
-      mbar_arrive(tempty_bar(acc));
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (CG == 2)
+          mbar_arrive_cluster(release_bar0 + 8u * acc);
+        else
+          mbar_arrive(release_bar0 + 8u * acc);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (CG == 2)
+    cluster_sync_all();  // neither CTA leaves while its peer may still touch its shared memory
+  else
+    __syncthreads();
   tc_fence_after_sync();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, Plan::kTmemCols);
+    tmem_dealloc<CG>(tmem_base, Plan::kTmemCols);
   }
 }
 
