@@ -294,16 +294,39 @@ def main(argv=None):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     override = json.loads(args.config) if args.config else None
     kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu, request=override)
+    # The split-K tail needs caller scratch; allocated once here, outside the timed region.
+    ws_bytes = tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, w.out, w.bias_relu, override)
+    ws = tlg.tlg_workspace(ws_bytes, device=dev) if ws_bytes > 0 else None
+    plain_name = ("tlg_gemm_bias_relu_f16" if w.bias_relu else
+                  ("tlg_gemm_f16f16" if w.out == "f16" else "tlg_gemm_f16f32"))
+    use_ex = ws is not None or override is not None
+    entry = "tlg_gemm_ex" if use_ex else plain_name
 
-    def step():
-        if override:
-            tlg.tlg_gemm_ex(dA, dB, dbias, dC, out=w.out, config=override, stream=stream)
-        elif w.bias_relu:
+    def plain_step():
+        if w.bias_relu:
             tlg.tlg_gemm_bias_relu_f16(dA, dB, dbias, dC, stream=stream)
         elif w.out == "f16":
             tlg.tlg_gemm_f16f16(dA, dB, dC, stream=stream)
         else:
             tlg.tlg_gemm_f16f32(dA, dB, dC, stream=stream)
+
+    def step():
+        if use_ex:
+            tlg.tlg_gemm_ex(dA, dB, dbias, dC, out=w.out, config=override, workspace=ws, stream=stream)
+        else:
+            plain_step()
+
+    def timed(fn, n):
+        """Per-step device milliseconds of n calls, each after an untimed L2 flush."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for i in range(n):
+            flush.fill_(float(i))  # untimed: evicts A, B and C from L2
+            starts[i].record(stream)
+            fn()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        return [s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)]
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -313,25 +336,30 @@ def main(argv=None):
     if rc != 0:
         raise SystemExit(f"device error word {code:#x} during warm-up")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     clocks = ClockSampler(nvsmi_id(dev))
     clocks.start()
     barrier(world)
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.fill_(float(i))  # untimed: evicts A, B and C from L2
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
+    per_step_ms = timed(step, args.steps)
     barrier(world)
     clk = clocks.stop()
-    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     gemm_ms = sum(per_step_ms)
     rc, code = tlg.tlg_device_error(clear=True)
     if rc != 0:
         raise SystemExit(f"device error word {code:#x} during the timed steps")
+
+    # The same steps through the plain entry point (no workspace), for comparison.
+    plain = None
+    if use_ex and override is None:
+        for _ in range(args.warmup):
+            flush.fill_(1.0)
+            plain_step()
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        plain_ms = max_over_ranks(sum(timed(plain_step, args.steps)), world)
+        barrier(world)
+        plain = {"call": plain_name, "value": w.flops * args.steps * world / (plain_ms * 1e-3) / 1e12,
+                 "unit": UNIT, "ms_per_step": plain_ms / args.steps}
 
     max_ms = max_over_ranks(gemm_ms, world)
     total_flops = w.flops * args.steps * world
@@ -403,8 +431,8 @@ def main(argv=None):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": workload_config(w, kcfg),
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "config": dict(workload_config(w, kcfg), entry_point=entry, workspace_bytes=ws_bytes),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "plain_entry_point": plain,
         "gpu_launches": args.steps,
         "clocks": clk,
         "per_step_ms": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),

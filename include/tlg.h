@@ -45,6 +45,7 @@
 #ifndef TLG_H
 #define TLG_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -106,11 +107,16 @@ typedef enum tlg_epilogue { TLG_EPI_NONE = 0, TLG_EPI_BIAS_RELU = 1 } tlg_epilog
  * Kernel configuration.  Zero in any field means "choose for me" (the
  * library's per-shape table, the analogue of the pages' cached tuned
  * configurations: "tilelang operator-compilation walkthrough" section 5.3).
- *   block_n     : output tile width per CTA, 64, 128 or 256 columns
- *   stages      : depth of the shared-memory operand ring, 2..8
+ *   block_n     : output tile width, 64, 128 or 256 columns
+ *   stages      : depth of the shared-memory operand ring (fixed per tile shape)
  *   cta_group   : 1 (one SM per 128-row tile) or 2 (an SM pair per 256-row tile)
  *   raster_group: number of tile rows walked together for L2 reuse, 1..64
  *   max_ctas    : cap on resident CTAs (0 = one per SM)
+ *   split_k     : 0 or 1 = every tile whole; 2..16 = the tiles left over
+ *                 after the last full wave are cut into that many k-slices
+ *                 (needs a workspace).  The automatic choice does not split:
+ *                 on a B200 under its power cap a split tail measured no
+ *                 faster at 4096^3 and slower at 1024^3.
  * A combination the library does not provide gives TLG_ERR_UNSUPPORTED.
  */
 typedef struct tlg_config {
@@ -119,13 +125,30 @@ typedef struct tlg_config {
     int32_t cta_group;
     int32_t raster_group;
     int32_t max_ctas;
+    int32_t split_k;
 } tlg_config;
 
 /*
  * The three entry points above in one call, with an explicit configuration
- * (NULL = automatic).  bias must be NULL unless epilogue is
- * TLG_EPI_BIAS_RELU, and the bias epilogue needs out == TLG_OUT_F16.
- * Same arguments, ownership and errors as above.
+ * (NULL = automatic) and an optional workspace.  bias must be NULL unless
+ * epilogue is TLG_EPI_BIAS_RELU, and the bias epilogue needs
+ * out == TLG_OUT_F16.  Same arguments, ownership and errors as above.
+ *
+ * Workspace (split-K tail): when the tile count leaves the last wave of SMs
+ * partly idle, the leftover tiles can be cut along K into slices that run
+ * concurrently; each slice writes an fp32 partial sum to the workspace and the
+ * last slice to finish adds all partials in slice order (so the result does
+ * not depend on timing) and writes C.  `workspace` is caller-owned device
+ * memory, 256-byte aligned, not overlapping A, B, C or the bias;
+ * tlg_gemm_workspace_size() gives the bytes a configuration needs (at most
+ * about 20 MB on a B200 for any shape: the tail holds fewer slices than
+ * there are SMs).  Its first 4 KB hold counters
+ * that must be ZERO before the first call (e.g. cudaMemsetAsync once); every
+ * completed call leaves them zero again.  Calls that overlap in time (other
+ * streams) must not share a workspace.  After a TLG_ERR_TIMEOUT report the
+ * counters may be non-zero: clear them again.  NULL or too small a workspace
+ * with split_k >= 2 is TLG_ERR_INVALID_ARG; without a split the workspace is
+ * not touched.
  */
 tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K,
                        const void *A, int64_t lda,
@@ -134,7 +157,17 @@ tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K,
                        void *C, int64_t ldc,
                        tlg_out out, tlg_epilogue epilogue,
                        const tlg_config *config,
+                       void *workspace, size_t workspace_bytes,
                        void *stream);
+
+/*
+ * Workspace bytes tlg_gemm_ex would use for this shape and configuration
+ * (NULL = automatic) when given enough; 0 when every tile runs whole.
+ * No kernel is launched; the only CUDA calls read device attributes.
+ */
+tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
+                                   tlg_epilogue epilogue, const tlg_config *config,
+                                   size_t *bytes);
 
 /*
  * Resolve a configuration for this shape.  On input *config (never NULL)

@@ -34,15 +34,20 @@ class Padded:
     def ptr(self):
         return self.buf.data_ptr() + self.ld * self.buf.element_size()
 
-    def guard_intact(self) -> bool:
+    def guard_changes(self):
+        """Buffer positions (row, col) outside the matrix whose poison was overwritten."""
         bits = self.buf.view(torch.int16 if self.dtype == torch.float16 else torch.int32)
         mask = torch.ones_like(bits, dtype=torch.bool)
         mask[1:1 + self.rows, :self.cols] = False
-        return bool((bits[mask] == self.poison).all().item())
+        bad = mask & (bits != self.poison)
+        return [tuple(x) for x in bad.nonzero().tolist()[:8]]
+
+    def guard_intact(self) -> bool:
+        return not self.guard_changes()
 
 
 def gemm_padded(lib, A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None, out: str,
-                config: dict | None = None, extra=(0, 0, 0), stream=None):
+                config: dict | None = None, extra=(0, 0, 0), stream=None, workspace=None):
     """Run one GEMM through tlg_gemm_ex on padded operands; returns (C as float64 numpy, guards ok)."""
     import ctypes
 
@@ -65,8 +70,24 @@ def gemm_padded(lib, A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None
                          pbias.data_ptr() if pbias is not None else None, pc.ptr(), pc.ld,
                          tlg.TLG_OUT_F32 if out == "f32" else tlg.TLG_OUT_F16,
                          tlg.TLG_EPI_BIAS_RELU if bias is not None else tlg.TLG_EPI_NONE,
-                         ctypes.byref(cfg) if cfg is not None else None, st)
+                         ctypes.byref(cfg) if cfg is not None else None,
+                         workspace.data_ptr() if workspace is not None else None,
+                         workspace.numel() if workspace is not None else 0, st)
     if rc != 0:
         raise tlg.TlgError(rc, "tlg_gemm_ex")
     torch.cuda.synchronize()
-    return pc.view.double().cpu().numpy(), pa.guard_intact() and pb.guard_intact() and pc.guard_intact()
+    changes = {name: b.guard_changes() for name, b in (("A", pa), ("B", pb), ("C", pc))}
+    return pc.view.double().cpu().numpy(), GuardReport(changes)
+
+
+class GuardReport:
+    """Truthy when no guard element changed; its repr names the changed positions."""
+
+    def __init__(self, changes):
+        self.changes = {k: v for k, v in changes.items() if v}
+
+    def __bool__(self):
+        return not self.changes
+
+    def __repr__(self):
+        return f"guard changes (buffer row, col) {self.changes}"

@@ -14,8 +14,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lib_path():
-    from tiled_dense_gemm_tlg_b200 import build
-    return build.build()
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location(
+        "tlg_build", os.path.join(ROOT, "tiled_dense_gemm_tlg_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
 
 
 def header_functions():
@@ -71,7 +76,10 @@ def test_host_side_rejections_need_no_gpu(lib_path):
     assert f(8, 8, 8, A, 8, A, 8, A + 64, 8, None) == tlg.TLG_ERR_INVALID_ARG  # C overlaps A
     assert f(0, 8, 8, None, 8, None, 8, None, 8, None) == tlg.TLG_OK  # empty: nothing to do
     assert lib.tlg_gemm_bias_relu_f16(8, 8, 8, A, 8, A, 8, None, A * 2, 8, None) == tlg.TLG_ERR_INVALID_ARG
-    assert lib.tlg_gemm_ex(8, 8, 8, A, 8, A, 8, A * 3, A * 2, 8, 0, 1, None, None) == tlg.TLG_ERR_UNSUPPORTED
+    assert lib.tlg_gemm_ex(8, 8, 8, A, 8, A, 8, A * 3, A * 2, 8, 0, 1, None, None, 0, None) == tlg.TLG_ERR_UNSUPPORTED
+    # workspace must be 256-byte aligned and must not overlap C
+    assert lib.tlg_gemm_ex(8, 8, 8, A, 8, A, 8, None, A * 2, 8, 0, 0, None, A * 4 + 16, 4096, None) == tlg.TLG_ERR_ALIGNMENT
+    assert lib.tlg_gemm_ex(8, 8, 8, A, 8, A, 8, None, A * 2, 8, 0, 0, None, A * 2, 4096, None) == tlg.TLG_ERR_INVALID_ARG
     assert lib.tlg_selftest_timeout(0, None) == tlg.TLG_ERR_INVALID_ARG
 
 

@@ -18,8 +18,12 @@ pytestmark = pytest.mark.gpu
 SIZES = [1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 256, 257]
 OUTS = [("f32", False), ("f16", False), ("f16", True)]
 WIDTHS = [64, 128, 256]
-# every tile shape the library builds: (CTAs per tile, tile width)
-TILES = [(1, 64), (1, 128), (1, 256), (2, 128), (2, 256)]
+# every kernel variant the library builds: (CTAs per tile, tile width, ring stages)
+TILES = [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6)]
+
+
+def tile_cfg(tile):
+    return {"cta_group": tile[0], "block_n": tile[1], "stages": tile[2]}
 
 
 @pytest.fixture(scope="module")
@@ -48,9 +52,8 @@ def edge_cases():
 @pytest.mark.parametrize("M,N,K,out,bias_relu,tile", edge_cases())
 def test_ragged_edges(lib, M, N, K, out, bias_relu, tile):
     A, B, bias = wl.make_operands(M, N, K, "uniform", bias=bias_relu, seed=M * 1000003 + N * 1009 + K)
-    cfg = {"cta_group": tile[0], "block_n": tile[1]}
-    got, guards = gemm_padded(lib, A, B, bias, out, config=cfg, extra=(8, 8, 4))
-    assert guards, "a write landed outside M x N, or padding was modified"
+    got, guards = gemm_padded(lib, A, B, bias, out, config=tile_cfg(tile), extra=(8, 8, 4))
+    assert guards, f"a write landed outside M x N, or padding was modified: {guards!r}"
     ref = oracle.gemm(A, B, bias=bias, relu=bias_relu, threads=4)
     assert np.isfinite(got).all(), "NaN padding leaked into the product"
     ok, worst, idx = oracle.within_tolerance(got, ref, out)
@@ -62,23 +65,22 @@ def test_ragged_edges(lib, M, N, K, out, bias_relu, tile):
 def test_every_tile_on_multi_tile_ragged_shape(lib, tile, out, bias_relu):
     M, N, K = 700, 520, 1000  # several tiles each way, ragged in M, N and K, many k-blocks
     A, B, bias = wl.make_operands(M, N, K, "normal025", bias=bias_relu, seed=5)
-    cfg = {"cta_group": tile[0], "block_n": tile[1]}
-    got, guards = gemm_padded(lib, A, B, bias, out, config=cfg, extra=(8, 16, 8))
-    assert guards
+    got, guards = gemm_padded(lib, A, B, bias, out, config=tile_cfg(tile), extra=(8, 16, 8))
+    assert guards, repr(guards)
     ref = oracle.gemm(A, B, bias=bias, relu=bias_relu)
     ok, worst, idx = oracle.within_tolerance(got, ref, out)
     assert ok, f"worst err/bound {worst:.3g} at {idx}"
 
 
-@pytest.mark.parametrize("tile", [(1, 128), (2, 256)])
+@pytest.mark.parametrize("tile", [(1, 128, 6), (2, 256, 6)])
 @pytest.mark.parametrize("raster_group,max_ctas", [(1, 0), (3, 0), (64, 0), (8, 2), (8, 7)])
 def test_scheduler_variants(lib, tile, raster_group, max_ctas):
     # fewer CTAs than tiles makes each CTA loop over many tiles and both TMEM accumulators
     M, N, K = 1100, 900, 333
     A, B, _ = wl.make_operands(M, N, K, "uniform", seed=6)
-    cfg = {"cta_group": tile[0], "block_n": tile[1], "raster_group": raster_group, "max_ctas": max_ctas}
+    cfg = dict(tile_cfg(tile), raster_group=raster_group, max_ctas=max_ctas)
     got, guards = gemm_padded(lib, A, B, None, "f32", config=cfg)
-    assert guards
+    assert guards, repr(guards)
     ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B), "f32")
     assert ok, f"worst err/bound {worst:.3g} at {idx}"
 

@@ -102,15 +102,15 @@ def test_integer_inputs_are_bit_exact(tlg, name):
         assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), want)
 
 
-@pytest.mark.parametrize("tile", [(1, 64), (1, 128), (1, 256), (2, 128), (2, 256)])
+@pytest.mark.parametrize("tile", [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6)])
 def test_every_tile_on_the_bias_relu_workload(tlg, tile):
-    # the full-size bias+ReLU workload under each tile shape the library builds
+    # the full-size bias+ReLU workload under each kernel variant the library builds
     w = wl.WORKLOADS["gemm_bias_relu_4096_f16"]
     A, B, bias = wl.workload_operands(w)
     C = tlg.tlg_gemm_ex(A.cuda(), B.cuda(), bias.cuda(), out="f16",
-                        config={"cta_group": tile[0], "block_n": tile[1]})
+                        config={"cta_group": tile[0], "block_n": tile[1], "stages": tile[2]})
     torch.cuda.synchronize()
-    er, ec = edge_positions(w.M, w.N, count=1024, seed=tile[0] * 7 + tile[1])
+    er, ec = edge_positions(w.M, w.N, count=1024, seed=sum(tile))
     check_positions(C, A, B, bias, w, er, ec)
 
 

@@ -32,7 +32,7 @@ LIB_PATH = os.path.join(_PKG, "libtlg.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"libtlg.so not found at {LIB_PATH}: build it with `python -m tiled_dense_gemm_tlg_b200.build` "
+        f"libtlg.so not found at {LIB_PATH}: build it with `python tiled_dense_gemm_tlg_b200/build.py` "
         "(there is no CPU fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -42,13 +42,14 @@ TLG_OUT_F32, TLG_OUT_F16 = 0, 1
 TLG_EPI_NONE, TLG_EPI_BIAS_RELU = 0, 1
 
 EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-            "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
+            "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
             "tlg_version")
 
 
 class tlg_config(ctypes.Structure):
     _fields_ = [("block_n", ctypes.c_int32), ("stages", ctypes.c_int32), ("cta_group", ctypes.c_int32),
-                ("raster_group", ctypes.c_int32), ("max_ctas", ctypes.c_int32)]
+                ("raster_group", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
+                ("split_k", ctypes.c_int32)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -58,8 +59,11 @@ _i64, _p, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
 _lib.tlg_gemm_f16f32.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p]
 _lib.tlg_gemm_f16f16.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p]
 _lib.tlg_gemm_bias_relu_f16.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _p]
+_sz = ctypes.c_size_t
 _lib.tlg_gemm_ex.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i32, _i32,
-                             ctypes.POINTER(tlg_config), _p]
+                             ctypes.POINTER(tlg_config), _p, _sz, _p]
+_lib.tlg_gemm_workspace_size.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config),
+                                         ctypes.POINTER(_sz)]
 _lib.tlg_choose_config.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config)]
 _lib.tlg_device_error.argtypes = [_i32, ctypes.POINTER(ctypes.c_uint32)]
 _lib.tlg_selftest_timeout.argtypes = [ctypes.c_uint32, _p]
@@ -67,7 +71,7 @@ _lib.tlg_status_string.argtypes = [_i32]
 _lib.tlg_status_string.restype = ctypes.c_char_p
 _lib.tlg_version.restype = ctypes.c_int32
 for _name in ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-              "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
+              "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
     getattr(_lib, _name).restype = _i32
 
 
@@ -162,8 +166,10 @@ def tlg_gemm_bias_relu_f16(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor,
 
 
 def tlg_gemm_ex(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None = None,
-                C: torch.Tensor | None = None, out: str = "f32", config: dict | None = None, stream=None):
-    """Explicit-configuration form; ``out`` is "f32" or "f16"; a bias selects the bias+ReLU epilogue."""
+                C: torch.Tensor | None = None, out: str = "f32", config: dict | None = None,
+                workspace: torch.Tensor | None = None, stream=None):
+    """Explicit-configuration form; ``out`` is "f32" or "f16"; a bias selects the bias+ReLU epilogue.
+    ``workspace``: optional device buffer (see ``tlg_workspace``) enabling the split-K tail."""
     M, N, K = _shapes(A, B)
     o = TLG_OUT_F32 if out == "f32" else TLG_OUT_F16
     C = _out(C, M, N, torch.float32 if o == TLG_OUT_F32 else torch.float16, A)
@@ -174,10 +180,29 @@ def tlg_gemm_ex(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None = No
     if config is not None:
         cfg = tlg_config(**{k: int(v) for k, v in config.items()})
     epi = TLG_EPI_BIAS_RELU if bias is not None else TLG_EPI_NONE
+    ws_ptr, ws_bytes = (None, 0)
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check(_lib.tlg_gemm_ex(M, N, K, pa, lda, pb, ldb, bias.data_ptr() if bias is not None else None,
                             pc, ldc, o, epi, ctypes.byref(cfg) if cfg is not None else None,
-                            _stream_handle(stream, A, B, C)), "tlg_gemm_ex")
+                            ws_ptr, ws_bytes, _stream_handle(stream, A, B, C)), "tlg_gemm_ex")
     return C
+
+
+def tlg_gemm_workspace_size(M: int, N: int, K: int, out: str = "f32", bias_relu: bool = False,
+                            config: dict | None = None) -> int:
+    cfg = tlg_config(**{k: int(v) for k, v in config.items()}) if config else None
+    n = ctypes.c_size_t(0)
+    _check(_lib.tlg_gemm_workspace_size(M, N, K, TLG_OUT_F32 if out == "f32" else TLG_OUT_F16,
+                                        TLG_EPI_BIAS_RELU if bias_relu else TLG_EPI_NONE,
+                                        ctypes.byref(cfg) if cfg is not None else None, ctypes.byref(n)),
+           "tlg_gemm_workspace_size")
+    return int(n.value)
+
+
+def tlg_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled device workspace of at least ``nbytes`` (torch's allocator; 256-byte aligned)."""
+    return torch.zeros(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
 
 
 def tlg_choose_config(M: int, N: int, K: int, out: str = "f32", bias_relu: bool = False,

@@ -1,6 +1,8 @@
 """Build libtlg.so in-tree with nvcc for sm_100a (B200).
 
-    python -m tiled_dense_gemm_tlg_b200.build [--force]
+    python tiled_dense_gemm_tlg_b200/build.py [--force]
+
+(Run it as a script: importing the package loads the library this builds.)
 
 The library is plain CUDA C++ behind the C interface in include/tlg.h; it does
 not link against torch.  The CUDA runtime is linked statically and the one

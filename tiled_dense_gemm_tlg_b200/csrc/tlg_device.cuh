@@ -59,6 +59,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test, but the thread may sleep in the instruction for up to
+// `suspend_ns` (it wakes as soon as the phase completes), so a waiting warp
+// neither spins nor burns issue slots while the main loop runs.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Longest sleep inside one try_wait of a bounded wait (10 ms); the time limit
+// and the abort flag are checked between sleeps.
+constexpr uint32_t kWaitSuspendNs = 10000000u;
+
 // Slow path of a bounded wait: spin until the phase of parity `parity`
 // completes, another role raises the CTA's abort flag, or `limit_ns` of wall
 // time pass.  On the time limit it records the role in the device error word
@@ -69,7 +89,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
                                             uint32_t role, uint32_t *err_word) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSuspendNs)) return true;
     if (abort_flag != nullptr && *abort_flag != 0u) return false;
     if (global_timer_ns() - t0 > limit_ns) {
       atomicOr(err_word, kErrTimeout | role);
@@ -114,6 +134,51 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
+}
+
+// 2-D tiled store of one box from shared memory to global memory, tracked in
+// this thread's bulk async-group; elements outside the tensor are skipped.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *tm, uint32_t src, int32_t x,
+                                             int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until at most N of this thread's bulk groups are still in flight.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Global accesses cached in L2 only, for data other CTAs of the same launch
+// write or read (L1 is not coherent across SMs).
+__device__ __forceinline__ void st_global_cg(float *ptr, float v) {
+  asm volatile("st.global.cg.f32 [%0], %1;" ::"l"(ptr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ float ld_global_cg(const float *ptr) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(ptr) : "memory");
+  return v;
 }
 
 // ------------------------------------------------------------------ clusters
@@ -274,6 +339,37 @@ __device__ __forceinline__ void tmem_load_32cols(uint32_t taddr, uint32_t (&r)[3
         "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
       :
       : "memory");
+}
+
+// Two 32-column loads (columns [col, col+32) and [col+32, col+64)) issued
+// back to back, then one wait.
+__device__ __forceinline__ void tmem_load_2x32cols(uint32_t taddr, uint32_t (&a)[32],
+                                                   uint32_t (&b)[32]) {
+#define TLG_LD32(R, ADDR)                                                                          \
+  asm volatile(                                                                                    \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32"                                                     \
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"                    \
+      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31},"          \
+      " [%32];"                                                                                    \
+      : "=r"(R[0]), "=r"(R[1]), "=r"(R[2]), "=r"(R[3]), "=r"(R[4]), "=r"(R[5]), "=r"(R[6]),        \
+        "=r"(R[7]), "=r"(R[8]), "=r"(R[9]), "=r"(R[10]), "=r"(R[11]), "=r"(R[12]), "=r"(R[13]),    \
+        "=r"(R[14]), "=r"(R[15]), "=r"(R[16]), "=r"(R[17]), "=r"(R[18]), "=r"(R[19]),              \
+        "=r"(R[20]), "=r"(R[21]), "=r"(R[22]), "=r"(R[23]), "=r"(R[24]), "=r"(R[25]),              \
+        "=r"(R[26]), "=r"(R[27]), "=r"(R[28]), "=r"(R[29]), "=r"(R[30]), "=r"(R[31])               \
+      : "r"(ADDR))
+#define TLG_FENCE32(R)                                                                             \
+  "+r"(R[0]), "+r"(R[1]), "+r"(R[2]), "+r"(R[3]), "+r"(R[4]), "+r"(R[5]), "+r"(R[6]), "+r"(R[7]),  \
+      "+r"(R[8]), "+r"(R[9]), "+r"(R[10]), "+r"(R[11]), "+r"(R[12]), "+r"(R[13]), "+r"(R[14]),     \
+      "+r"(R[15]), "+r"(R[16]), "+r"(R[17]), "+r"(R[18]), "+r"(R[19]), "+r"(R[20]), "+r"(R[21]),   \
+      "+r"(R[22]), "+r"(R[23]), "+r"(R[24]), "+r"(R[25]), "+r"(R[26]), "+r"(R[27]), "+r"(R[28]),   \
+      "+r"(R[29]), "+r"(R[30]), "+r"(R[31])
+  TLG_LD32(a, taddr);
+  TLG_LD32(b, taddr + 32);
+  // The wait names every destination register, so no use of them can move above it.
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : TLG_FENCE32(a) : : "memory");
+  asm volatile("" : TLG_FENCE32(b) : : "memory");
+#undef TLG_LD32
+#undef TLG_FENCE32
 }
 
 // ------------------------------------------------------------------ descriptors

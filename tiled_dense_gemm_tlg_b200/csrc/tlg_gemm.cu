@@ -1,10 +1,12 @@
 // Host side of libtlg: argument checks, TMA descriptor encoding, the per-shape
-// configuration table and the launches behind the C interface in tlg.h.
+// configuration table, the work schedule and the launches behind the C
+// interface in tlg.h.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdint>
 #include <mutex>
 
 #include "tlg.h"
@@ -16,6 +18,8 @@ using namespace tlg;
 
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
+constexpr size_t kCounterBytes = 4096;            // slice counters at the start of a workspace
+constexpr size_t kWorkspaceAlign = 256;
 
 struct DeviceInfo {
   bool probed = false;
@@ -84,7 +88,7 @@ void extent(const void *p, int64_t rows, int64_t cols, int64_t ld, int64_t esz, 
 
 bool overlaps(uintptr_t a0, uintptr_t a1, uintptr_t b0, uintptr_t b1) { return a0 < b1 && b0 < a1; }
 
-// --------------------------------------------------------------------------- configurations
+// --------------------------------------------------------------------------- kernel variants
 
 struct KernelCfg {
   int cta_group;
@@ -93,168 +97,229 @@ struct KernelCfg {
   double eff;  // fraction of the MMA peak one tile sustains (used to rank tile shapes)
 };
 
-// Tile shapes the library is built with.  A tile is 128*cta_group rows by
-// block_n columns; `stages` is the deepest operand ring that fits in 227 KB of
-// shared memory next to the barriers.  Per-CTA ring slot: 16 KB of A plus
-// 128*block_n/cta_group bytes of B.
+// Kernel variants the library is built with.  A tile is 128*cta_group rows by
+// block_n columns; `stages` is the depth of the operand ring (per-CTA slot:
+// 16 KB of A plus 128*block_n/cta_group bytes of B), as deep as fits in
+// 227 KB of shared memory next to 32 KB of output staging.
 // `eff` is measured: TFLOP/s of each shape on a B200 at M = N = K = 4096 and
 // 8192 after dividing out the wave count, relative to the 2 x 256 pair tile.
 constexpr KernelCfg kBuilt[] = {
     {1, 64, 8, 0.35}, {1, 128, 6, 0.60}, {1, 256, 4, 0.90}, {2, 128, 8, 0.60}, {2, 256, 6, 1.00}};
+constexpr int kNumBuilt = sizeof(kBuilt) / sizeof(kBuilt[0]);
 
-const KernelCfg *find_built(int cta_group, int block_n) {
-  for (const KernelCfg &k : kBuilt)
-    if (k.cta_group == cta_group && k.block_n == block_n) return &k;
-  return nullptr;
-}
-
-// Pick the tile shape with the fewest estimated SM-time units: whole waves of
-// tiles over the available CTAs (pairs), times the tile's work over its
-// sustained fraction of the MMA peak.  Narrow and single-SM tiles sustain less
-// because each 128-row MMA reads all of its A tile from shared memory for
-// every block_n columns it produces.
-void choose(int64_t M, int64_t N, int sms, tlg_config *c) {
-  double best = 0;
-  const KernelCfg *pick = &kBuilt[0];
-  for (const KernelCfg &k : kBuilt) {
-    const int64_t tile_m = 128 * k.cta_group;
-    const int64_t tiles = ((M + tile_m - 1) / tile_m) * ((N + k.block_n - 1) / k.block_n);
-    const int64_t units = sms / k.cta_group;
-    const int64_t waves = (tiles + units - 1) / units;
-    const double cost = static_cast<double>(waves) * tile_m * k.block_n / (k.cta_group * k.eff);
-    if (&k == &kBuilt[0] || cost < best * 0.999) {
-      best = cost;
-      pick = &k;
-    }
-  }
-  c->block_n = pick->block_n;
-  c->stages = pick->stages;
-  c->cta_group = pick->cta_group;
-  c->raster_group = 8;
-  c->max_ctas = 0;
-}
-
-tlg_status resolve_config(int64_t M, int64_t N, int sms, const tlg_config *req, tlg_config *out) {
-  choose(M, N, sms, out);
-  if (req == nullptr) return TLG_OK;
-  int cg = req->cta_group != 0 ? req->cta_group : out->cta_group;
-  int bn = req->block_n != 0 ? req->block_n : out->block_n;
-  const KernelCfg *k = find_built(cg, bn);
-  if (k == nullptr) {
-    // a width given alone may exist only for the other CTA-group size
-    if (req->cta_group == 0 && req->block_n != 0) {
-      cg = 3 - cg;
-      k = find_built(cg, bn);
-    }
-    if (k == nullptr) return TLG_ERR_UNSUPPORTED;
-  }
-  out->cta_group = cg;
-  out->block_n = bn;
-  out->stages = k->stages;
-  if (req->stages != 0 && req->stages != k->stages) return TLG_ERR_UNSUPPORTED;
-  if (req->raster_group != 0) {
-    if (req->raster_group < 1 || req->raster_group > 64) return TLG_ERR_UNSUPPORTED;
-    out->raster_group = req->raster_group;
-  }
-  if (req->max_ctas < 0) return TLG_ERR_UNSUPPORTED;
-  out->max_ctas = req->max_ctas;
-  return TLG_OK;
-}
-
-// --------------------------------------------------------------------------- launch
-
-bool encode_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
-               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estride[2] = {1, 1};
-  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims,
-                              strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
+// Per device and instantiation: kernel attributes set, co-resident work units.
 struct LaunchState {
-  bool attr_set = false;
-  int max_clusters = 0;  // co-resident clusters of this kernel (cta_group 2)
+  bool ready = false;
+  int units = 0;
 };
 
-// Launch one kernel instantiation: persistent grid of one CTA per SM (or one
-// cluster per SM pair, limited to the clusters that fit at once), capped by
-// the tile count and max_ctas.
 template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
-tlg_status launch_gemm(int dev, int sms, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                       const GemmParams &p, int64_t tiles, int max_ctas, cudaStream_t stream) {
+struct Variant {
   using Plan = SmemPlan<CG, BN, STAGES>;
-  auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU>;
-  static LaunchState state[kMaxDevices];
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Plan::kDynamicBytes;
-  cfg.stream = stream;
-  if (CG == 2) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+
+  static void fill_launch(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, cudaStream_t s) {
+    *cfg = {};
+    cfg->blockDim = dim3(kThreads, 1, 1);
+    cfg->dynamicSmemBytes = Plan::kDynamicBytes;
+    cfg->stream = s;
+    if (CG == 2) {
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg->attrs = attr;
+      cfg->numAttrs = 1;
+    }
   }
-  {
+
+  // Work units (CTAs, or CTA pairs) that can be resident at once: one per SM,
+  // or the number of 2-CTA clusters the occupancy calculator admits.
+  static tlg_status units(int dev, int sms, int *out) {
+    static LaunchState state[kMaxDevices];
+    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU>;
     std::lock_guard<std::mutex> lock(g_mutex);
     LaunchState &st = state[dev];
-    if (!st.attr_set) {
+    if (!st.ready) {
       if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Plan::kDynamicBytes) != cudaSuccess) {
         cudaGetLastError();
         return TLG_ERR_CUDA;
       }
+      int n = sms;
       if (CG == 2) {
+        cudaLaunchConfig_t cfg;
+        cudaLaunchAttribute attr[1];
+        fill_launch(&cfg, attr, nullptr);
         cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-        int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
           cudaGetLastError();
           return TLG_ERR_CUDA;
         }
-        st.max_clusters = n;
       }
-      st.attr_set = true;
+      st.units = n;
+      st.ready = true;
+    }
+    *out = st.units;
+    return TLG_OK;
+  }
+
+  static tlg_status launch(int units, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                           const CUtensorMap &tmC, const GemmParams &p, cudaStream_t s) {
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    fill_launch(&cfg, attr, s);
+    cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU>, tmA, tmB, tmC, p);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return TLG_ERR_CUDA;
+    }
+    return TLG_OK;
+  }
+};
+
+struct VariantFns {
+  tlg_status (*units)(int, int, int *);
+  tlg_status (*launch)(int, const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
+                       const GemmParams &, cudaStream_t);
+};
+
+#define TLG_FNS(CG, BN, ST, F16, BR) \
+  VariantFns { Variant<CG, BN, ST, F16, BR>::units, Variant<CG, BN, ST, F16, BR>::launch }
+#define TLG_VARIANT(CG, BN, ST) \
+  { TLG_FNS(CG, BN, ST, false, false), TLG_FNS(CG, BN, ST, true, false), TLG_FNS(CG, BN, ST, true, true) }
+
+// [variant, same order as kBuilt][f32 | f16 | f16 bias+ReLU]
+const VariantFns kVariantFns[kNumBuilt][3] = {TLG_VARIANT(1, 64, 8), TLG_VARIANT(1, 128, 6),
+                                              TLG_VARIANT(1, 256, 4), TLG_VARIANT(2, 128, 8),
+                                              TLG_VARIANT(2, 256, 6)};
+#undef TLG_VARIANT
+#undef TLG_FNS
+
+const VariantFns &fns_for(int idx, bool f16, bool bias_relu) {
+  return kVariantFns[idx][!f16 ? 0 : (bias_relu ? 2 : 1)];
+}
+
+// --------------------------------------------------------------------------- schedule
+
+// How one launch spreads the tiles over its work units.
+struct Schedule {
+  int64_t tiles = 0;
+  int units = 0;  // grid size in work units
+  int dp_tiles = 0;
+  int split = 1;
+  int tail_items = 0;
+  size_t workspace = 0;  // bytes needed (0 without a split tail)
+  double cost = 0;       // k-blocks on the longest unit's path
+};
+
+size_t split_workspace_bytes(int tail_items, int cta_group, int block_n) {
+  return kCounterBytes +
+         static_cast<size_t>(tail_items) * cta_group * 4 * 32 * block_n * sizeof(float);
+}
+
+// Plan for `split` k-slices per tail tile (1 = every tile whole, one after the
+// other on `resident` units).  A split keeps ceil(T/U)-1 whole waves and cuts
+// the remaining tiles so that the last wave is as short as a slice.
+bool plan(int64_t tiles, int resident, int num_kb, int split, int cta_group, int block_n,
+          Schedule *s) {
+  s->tiles = tiles;
+  if (split <= 1) {
+    s->units = static_cast<int>(std::min<int64_t>(resident, tiles));
+    s->dp_tiles = static_cast<int>(tiles);
+    s->split = 1;
+    s->tail_items = 0;
+    s->workspace = 0;
+    s->cost = static_cast<double>((tiles + s->units - 1) / s->units) * num_kb;
+    return true;
+  }
+  if (split > num_kb) return false;
+  const int64_t full = tiles / resident;
+  const int64_t rem = full > 0 ? tiles % resident : tiles;
+  if (rem == 0 || rem * split > resident) return false;
+  s->units = full > 0 ? resident : static_cast<int>(rem * split);
+  s->dp_tiles = static_cast<int>(full * resident);
+  s->split = split;
+  s->tail_items = static_cast<int>(rem * split);
+  s->workspace = split_workspace_bytes(s->tail_items, cta_group, block_n);
+  // The slice runs first; its partial-sum traffic hides behind the next whole
+  // tile unless there is none, and then it costs about 2 + split k-blocks.
+  const double slice = static_cast<double>((num_kb + split - 1) / split);
+  s->cost = static_cast<double>(full) * num_kb + slice + (full > 0 ? 0.5 : 2.0 + split);
+  return true;
+}
+
+struct Resolved {
+  tlg_config cfg;
+  int idx;
+  Schedule sched;
+};
+
+// Choose (or check) the kernel variant and the schedule.  Shapes are ranked by
+// k-blocks on the critical path times the per-k-block time of the tile (tile
+// area over its sustained fraction of the MMA peak, per SM).
+tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, bool bias_relu,
+                   const tlg_config *req, size_t ws_bytes, Resolved *out) {
+  const int num_kb = static_cast<int>((K + kBK - 1) / kBK);
+  tlg_config r = {};
+  if (req != nullptr) r = *req;
+  if (r.raster_group < 0 || r.raster_group > 64 || r.max_ctas < 0 || r.split_k < 0 ||
+      r.split_k > 16 || r.stages < 0 || r.block_n < 0 || r.cta_group < 0)
+    return TLG_ERR_UNSUPPORTED;
+  double best_cost = 0;
+  bool found = false;
+  bool shape_exists = false;
+  for (int i = 0; i < kNumBuilt; ++i) {
+    const KernelCfg &k = kBuilt[i];
+    if (r.cta_group != 0 && r.cta_group != k.cta_group) continue;
+    if (r.block_n != 0 && r.block_n != k.block_n) continue;
+    if (r.stages != 0 && r.stages != k.stages) continue;
+    shape_exists = true;
+    int resident = 0;
+    const tlg_status us = fns_for(i, f16, bias_relu).units(dev, sms, &resident);
+    if (us != TLG_OK) return us;
+    if (r.max_ctas > 0) resident = std::max(1, std::min(resident, r.max_ctas / k.cta_group));
+    const int64_t tile_m = 128 * k.cta_group;
+    const int64_t tiles = ((M + tile_m - 1) / tile_m) * ((N + k.block_n - 1) / k.block_n);
+    // Automatic choice (split_k == 0) runs every tile whole: measured on a
+    // B200 the split tail gained nothing at 4096^3 (1353 vs 1349 TFLOP/s; under
+    // the 1000 W cap the SMs idle in a partial last wave let the busy ones
+    // clock higher) and lost at 1024^3, where its fix-up is exposed.
+    Schedule sch;
+    (void)ws_bytes;
+    if (!plan(tiles, resident, num_kb, r.split_k == 0 ? 1 : r.split_k, k.cta_group, k.block_n, &sch))
+      continue;
+    const double cost = sch.cost * static_cast<double>(tile_m * k.block_n) / (k.cta_group * k.eff);
+    if (!found || cost < best_cost * 0.999) {
+      found = true;
+      best_cost = cost;
+      out->idx = i;
+      out->sched = sch;
+      out->cfg.cta_group = k.cta_group;
+      out->cfg.block_n = k.block_n;
+      out->cfg.stages = k.stages;
     }
   }
-  int64_t units = CG == 2 ? state[dev].max_clusters : sms;
-  if (max_ctas > 0) units = std::min<int64_t>(units, std::max(1, max_ctas / CG));
-  units = std::min<int64_t>(units, tiles);
-  cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, p);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return TLG_ERR_CUDA;
-  }
+  if (!shape_exists || !found) return TLG_ERR_UNSUPPORTED;
+  out->cfg.raster_group = r.raster_group != 0 ? r.raster_group : 8;
+  out->cfg.max_ctas = r.max_ctas;
+  out->cfg.split_k = out->sched.split;
   return TLG_OK;
 }
 
-template <bool OUT_F16, bool BIAS_RELU>
-tlg_status dispatch(int dev, int sms, const tlg_config &c, const CUtensorMap &tmA,
-                    const CUtensorMap &tmB, const GemmParams &p, cudaStream_t s) {
-  const int64_t tile_m = 128 * c.cta_group;
-  const int64_t tiles = ((p.M + tile_m - 1) / tile_m) * ((p.N + c.block_n - 1) / c.block_n);
-  const int mc = c.max_ctas;
-  if (c.cta_group == 1) {
-    switch (c.block_n) {
-      case 256: return launch_gemm<1, 256, 4, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
-      case 128: return launch_gemm<1, 128, 6, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
-      case 64: return launch_gemm<1, 64, 8, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
-      default: return TLG_ERR_UNSUPPORTED;
-    }
-  }
-  switch (c.block_n) {
-    case 256: return launch_gemm<2, 256, 6, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
-    case 128: return launch_gemm<2, 128, 8, OUT_F16, BIAS_RELU>(dev, sms, tmA, tmB, p, tiles, mc, s);
-    default: return TLG_ERR_UNSUPPORTED;
-  }
+// --------------------------------------------------------------------------- launch
+
+bool encode_2d(CUtensorMap *tm, CUtensorMapDataType dtype, const void *base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = g_encode(tm, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 template <bool OUT_F16, bool BIAS_RELU>
@@ -272,10 +337,10 @@ tlg_status launch_fill(void *C, int64_t ldc, const void *bias, int M, int N, cud
   return TLG_OK;
 }
 
-tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
-                     int64_t ldb, const void *bias, void *C, int64_t ldc, tlg_out out,
-                     tlg_epilogue epi, const tlg_config *req, void *stream) {
-  // ---- host-only checks first: nothing below touches the GPU until they pass
+// Host-only argument checks shared by every entry point; nothing here touches the GPU.
+tlg_status check_args(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
+                      int64_t ldb, const void *bias, const void *C, int64_t ldc, tlg_out out,
+                      tlg_epilogue epi) {
   if (out != TLG_OUT_F32 && out != TLG_OUT_F16) return TLG_ERR_INVALID_ARG;
   if (epi != TLG_EPI_NONE && epi != TLG_EPI_BIAS_RELU) return TLG_ERR_INVALID_ARG;
   if (epi == TLG_EPI_BIAS_RELU && out != TLG_OUT_F16) return TLG_ERR_UNSUPPORTED;
@@ -307,6 +372,32 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
     const uintptr_t s0 = reinterpret_cast<uintptr_t>(bias);
     if (overlaps(c0, c1, s0, s0 + static_cast<uintptr_t>(2 * N))) return TLG_ERR_INVALID_ARG;
   }
+  return TLG_OK;
+}
+
+// ws/ws_bytes: scratch for the split-K tail (nullptr/0: none).
+tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
+                     int64_t ldb, const void *bias, void *C, int64_t ldc, tlg_out out,
+                     tlg_epilogue epi, const tlg_config *req, void *ws, size_t ws_bytes,
+                     void *stream) {
+  const tlg_status hs = check_args(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epi);
+  if (hs != TLG_OK || M == 0 || N == 0) return hs;
+  const int64_t osz = out == TLG_OUT_F32 ? 4 : 2;
+  if (ws == nullptr) ws_bytes = 0;
+  if (ws != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(ws) % kWorkspaceAlign) != 0) return TLG_ERR_ALIGNMENT;
+    uintptr_t c0, c1;
+    extent(C, M, N, ldc, osz, &c0, &c1);
+    const uintptr_t w0 = reinterpret_cast<uintptr_t>(ws);
+    if (overlaps(c0, c1, w0, w0 + ws_bytes)) return TLG_ERR_INVALID_ARG;
+    if (K > 0) {
+      uintptr_t a0, a1, b0, b1;
+      extent(A, M, K, lda, 2, &a0, &a1);
+      extent(B, K, N, ldb, 2, &b0, &b1);
+      if (overlaps(w0, w0 + ws_bytes, a0, a1) || overlaps(w0, w0 + ws_bytes, b0, b1))
+        return TLG_ERR_INVALID_ARG;
+    }
+  }
 
   // ---- device checks
   int dev = 0;
@@ -317,10 +408,7 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
   if (K > 0 && (!device_accessible(A, dev) || !device_accessible(B, dev)))
     return TLG_ERR_INVALID_ARG;
   if (bias != nullptr && !device_accessible(bias, dev)) return TLG_ERR_INVALID_ARG;
-
-  tlg_config cfg;
-  const tlg_status cs = resolve_config(M, N, info.sm_count, req, &cfg);
-  if (cs != TLG_OK) return cs;
+  if (ws != nullptr && !device_accessible(ws, dev)) return TLG_ERR_INVALID_ARG;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool f16 = out == TLG_OUT_F16;
@@ -331,23 +419,54 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
     return launch_fill<true, false>(C, ldc, bias, int(M), int(N), s);
   }
 
-  CUtensorMap tmA, tmB;
-  if (!encode_2d(&tmA, A, uint64_t(K), uint64_t(M), uint64_t(lda) * 2, kBK, kBM) ||
-      !encode_2d(&tmB, B, uint64_t(N), uint64_t(K), uint64_t(ldb) * 2, 64, kBK))
+  Resolved rv;
+  const tlg_status rs = resolve(dev, info.sm_count, M, N, K, f16, br, req, ws_bytes, &rv);
+  if (rs != TLG_OK) return rs;
+  if (rv.sched.workspace > ws_bytes) return TLG_ERR_INVALID_ARG;  // a forced split needs scratch
+
+  // A: K x M boxes of 64 x 128; B: N x K boxes of 64 x 64; C: 32-row boxes of 128 bytes.
+  CUtensorMap tmA, tmB, tmC;
+  const CUtensorMapDataType c_type =
+      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (!encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, A, uint64_t(K), uint64_t(M),
+                 uint64_t(lda) * 2, kBK, kBM) ||
+      !encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, B, uint64_t(N), uint64_t(K),
+                 uint64_t(ldb) * 2, 64, kBK) ||
+      !encode_2d(&tmC, c_type, C, uint64_t(N), uint64_t(M), uint64_t(ldc) * osz,
+                 uint32_t(128 / osz), 32))
     return TLG_ERR_CUDA;
 
   GemmParams p;
-  p.C = C;
   p.bias = static_cast<const __half *>(bias);
+  p.C = C;
   p.ldc = ldc;
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
-  p.raster_group = cfg.raster_group;
+  p.raster_group = rv.cfg.raster_group;
+  p.n_aligned = (N * osz) % 16 == 0 ? 1 : 0;
   p.limit_ns = kWaitLimitNs;
-  if (!f16) return dispatch<false, false>(dev, info.sm_count, cfg, tmA, tmB, p, s);
-  if (br) return dispatch<true, true>(dev, info.sm_count, cfg, tmA, tmB, p, s);
-  return dispatch<true, false>(dev, info.sm_count, cfg, tmA, tmB, p, s);
+  p.dp_tiles = rv.sched.dp_tiles;
+  p.split = rv.sched.split;
+  p.tail_items = rv.sched.tail_items;
+  p.counters = static_cast<uint32_t *>(ws);
+  p.ws = ws != nullptr ? reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes)
+                       : nullptr;
+  return fns_for(rv.idx, f16, br).launch(rv.sched.units, tmA, tmB, tmC, p, s);
+}
+
+tlg_status resolve_public(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_epilogue epilogue,
+                          const tlg_config *req, size_t ws_bytes, Resolved *rv) {
+  if (out != TLG_OUT_F32 && out != TLG_OUT_F16) return TLG_ERR_INVALID_ARG;
+  if (epilogue != TLG_EPI_NONE && epilogue != TLG_EPI_BIAS_RELU) return TLG_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0) return TLG_ERR_INVALID_ARG;
+  int dev = 0;
+  DeviceInfo info;
+  const tlg_status ds = current_device(&dev, &info);
+  if (ds != TLG_OK) return ds;
+  return resolve(dev, info.sm_count, std::max<int64_t>(M, 1), std::max<int64_t>(N, 1),
+                 std::max<int64_t>(K, 1), out == TLG_OUT_F16, epilogue == TLG_EPI_BIAS_RELU, req,
+                 ws_bytes, rv);
 }
 
 }  // namespace
@@ -357,13 +476,13 @@ extern "C" {
 tlg_status tlg_gemm_f16f32(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                            const void *B, int64_t ldb, float *C, int64_t ldc, void *stream) {
   return gemm_impl(M, N, K, A, lda, B, ldb, nullptr, C, ldc, TLG_OUT_F32, TLG_EPI_NONE, nullptr,
-                   stream);
+                   nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_f16f16(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                            const void *B, int64_t ldb, void *C, int64_t ldc, void *stream) {
   return gemm_impl(M, N, K, A, lda, B, ldb, nullptr, C, ldc, TLG_OUT_F16, TLG_EPI_NONE, nullptr,
-                   stream);
+                   nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_bias_relu_f16(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
@@ -371,26 +490,39 @@ tlg_status tlg_gemm_bias_relu_f16(int64_t M, int64_t N, int64_t K, const void *A
                                   int64_t ldc, void *stream) {
   if (bias == nullptr && M > 0 && N > 0) return TLG_ERR_INVALID_ARG;
   return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, TLG_OUT_F16, TLG_EPI_BIAS_RELU, nullptr,
-                   stream);
+                   nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
                        int64_t ldb, const void *bias, void *C, int64_t ldc, tlg_out out,
-                       tlg_epilogue epilogue, const tlg_config *config, void *stream) {
-  return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, stream);
+                       tlg_epilogue epilogue, const tlg_config *config, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+  return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, workspace,
+                   workspace_bytes, stream);
+}
+
+tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
+                                   tlg_epilogue epilogue, const tlg_config *config, size_t *bytes) {
+  if (bytes == nullptr) return TLG_ERR_INVALID_ARG;
+  *bytes = 0;
+  if (M < 0 || N < 0 || K < 0) return TLG_ERR_INVALID_ARG;
+  if (M == 0 || N == 0 || K == 0) return TLG_OK;
+  Resolved rv;
+  const tlg_status rs = resolve_public(M, N, K, out, epilogue, config, SIZE_MAX, &rv);
+  if (rs != TLG_OK) return rs;
+  *bytes = rv.sched.workspace;
+  return TLG_OK;
 }
 
 tlg_status tlg_choose_config(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_epilogue epilogue,
                              tlg_config *config) {
-  (void)out;
-  (void)epilogue;
-  if (config == nullptr || M < 0 || N < 0 || K < 0) return TLG_ERR_INVALID_ARG;
-  int dev = 0;
-  DeviceInfo info;
-  const tlg_status ds = current_device(&dev, &info);
-  if (ds != TLG_OK) return ds;
+  if (config == nullptr) return TLG_ERR_INVALID_ARG;
+  Resolved rv;
   const tlg_config req = *config;
-  return resolve_config(M, N, info.sm_count, &req, config);
+  const tlg_status rs = resolve_public(M, N, K, out, epilogue, &req, SIZE_MAX, &rv);
+  if (rs != TLG_OK) return rs;
+  *config = rv.cfg;
+  return TLG_OK;
 }
 
 tlg_status tlg_device_error(int clear, uint32_t *code_out) {
@@ -432,15 +564,21 @@ tlg_status tlg_selftest_timeout(uint32_t limit_us, void *stream) {
 const char *tlg_status_string(tlg_status status) {
   switch (status) {
     case TLG_OK: return "TLG_OK";
-    case TLG_ERR_INVALID_ARG: return "TLG_ERR_INVALID_ARG: bad size, null or host pointer, ld too small, or overlapping output";
-    case TLG_ERR_ALIGNMENT: return "TLG_ERR_ALIGNMENT: pointers must be 16-byte aligned and row strides multiples of 16 bytes";
-    case TLG_ERR_UNSUPPORTED: return "TLG_ERR_UNSUPPORTED: device is not sm_100, size too large, or configuration not provided";
+    case TLG_ERR_INVALID_ARG:
+      return "TLG_ERR_INVALID_ARG: bad size, null or host pointer, ld too small, overlapping "
+             "buffers, or a workspace too small for the requested split";
+    case TLG_ERR_ALIGNMENT:
+      return "TLG_ERR_ALIGNMENT: pointers must be 16-byte aligned (the workspace 256-byte) and row "
+             "strides multiples of 16 bytes";
+    case TLG_ERR_UNSUPPORTED:
+      return "TLG_ERR_UNSUPPORTED: device is not sm_100, size too large, or configuration not "
+             "provided";
     case TLG_ERR_CUDA: return "TLG_ERR_CUDA: a CUDA call failed";
     case TLG_ERR_TIMEOUT: return "TLG_ERR_TIMEOUT: a kernel pipeline wait exceeded its time limit";
   }
   return "unknown tlg_status";
 }
 
-int32_t tlg_version(void) { return 100; }
+int32_t tlg_version(void) { return 200; }
 
 }  // extern "C"

@@ -15,8 +15,9 @@
 //                      Warp 1 also owns the TMEM allocation.
 //   warps 2-5          epilogue: tcgen05.ld of the accumulator, then bias,
 //                      ReLU and the output cast ("domestic-GPU TileLang
-//                      adoption", xdnf.cn/news/333523, section 4.2), and a
-//                      predicated store of the rows and columns inside M x N.
+//                      adoption", xdnf.cn/news/333523, section 4.2), staged in
+//                      shared memory and written by TMA bulk-tensor stores,
+//                      which clip the rows and columns outside M x N.
 //
 // CTAs are persistent (one per SM) and walk the tile list with a stride of
 // gridDim.x; consecutive tiles are grouped by `raster_group` row blocks so
@@ -24,29 +25,33 @@
 //
 // Ragged M, N and K need no special code in the main loop: the TMA unit fills
 // out-of-range elements of a box with zeros, so the last k-block adds 0 for
-// k >= K, and rows/columns beyond M/N are simply not stored.
+// k >= K, and the TMA store skips the rows/columns beyond M/N.
 #pragma once
 
 #include "tlg_device.cuh"
 
 namespace tlg {
 
-constexpr int kBM = 128;  // tile rows (TMEM lanes)
+constexpr int kBM = 128;  // tile rows per CTA (TMEM lanes)
 constexpr int kBK = 64;   // k-block: 64 fp16 = one 128-byte swizzle row
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 32 * (2 + kEpiWarps);  // producer warp, MMA warp, epilogue warps
+constexpr uint32_t kStageOutBytes = 32 * 128;   // one TMA store box: 32 rows x 128 bytes
 
 __device__ uint32_t g_device_error;
 
 // Shared-memory plan of one CTA.  CG CTAs (1 or 2) compute one tile of
 // 128*CG rows by BN columns; each CTA stages its own 128 rows of A and its own
-// BN/CG columns of B per k-block.
+// BN/CG columns of B per k-block, plus two 4 KB output boxes per epilogue warp.
 template <int CG, int BN, int STAGES>
 struct SmemPlan {
   static constexpr int kBNc = BN / CG;  // B columns held by one CTA
   static constexpr uint32_t kABytes = kBM * kBK * 2;
   static constexpr uint32_t kBBytes = kBK * kBNc * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kBarOffset = STAGES * kStageBytes;
+  static constexpr uint32_t kOutOffset = STAGES * kStageBytes;
+  static constexpr uint32_t kOutBytes = kEpiWarps * 2 * kStageOutBytes;
+  static constexpr uint32_t kBarOffset = kOutOffset + kOutBytes;
   static constexpr uint32_t kNumBars = 2 * STAGES + 4 + 1;  // full, empty, tmem full/empty x2, drain
   static constexpr uint32_t kMiscOffset = kBarOffset + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOffset + 16;
@@ -58,13 +63,63 @@ struct SmemPlan {
 };
 
 struct GemmParams {
-  void *C;
   const __half *bias;
+  void *C;       // used only for the ragged last column box when N is not 16-byte aligned
   int64_t ldc;
   int M, N, K;
   int raster_group;
+  int n_aligned;  // N * sizeof(out) is a multiple of 16: every box may go through TMA
   uint64_t limit_ns;
+  // Split-K tail (split > 1): tiles [dp_tiles, num_tiles) are each cut into
+  // `split` k-slices, tail_items = (num_tiles - dp_tiles) * split <= work units.
+  int dp_tiles;
+  int split;
+  int tail_items;
+  float *ws;           // fp32 partial sums of the tail slices
+  uint32_t *counters;  // per (tail tile, CTA of the group, epilogue warp): slices written so far
 };
+
+// One unit of work: a tile, or one k-slice of a tail tile.
+struct WorkItem {
+  int mb, nb;    // tile coordinates (in tiles)
+  int kb0, kb1;  // k-blocks [kb0, kb1)
+  int tail;      // index among the tail tiles, or -1 for a whole tile
+  int slice;
+};
+
+// Work list of one unit (a CTA, or a CTA pair): its tail slice first, if it
+// has one, then the whole tiles unit, unit + num_units, ... below dp_tiles.
+// Doing the slice first lets its partial-sum traffic run in the epilogue
+// while the next tile's main loop already runs.
+__device__ __forceinline__ int work_count(const GemmParams &p, int unit, int num_units) {
+  const int whole = p.dp_tiles > unit ? (p.dp_tiles - unit + num_units - 1) / num_units : 0;
+  return whole + (unit < p.tail_items ? 1 : 0);
+}
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int group, int &mb,
+                                            int &nb);
+
+__device__ __forceinline__ WorkItem work_item(const GemmParams &p, int k, int unit, int num_units,
+                                              int num_m, int num_n, int num_kb) {
+  WorkItem w;
+  const bool has_tail = unit < p.tail_items;
+  int t;
+  if (has_tail && k == 0) {
+    w.tail = unit / p.split;
+    w.slice = unit - w.tail * p.split;
+    t = p.dp_tiles + w.tail;
+    w.kb0 = static_cast<int>(static_cast<int64_t>(w.slice) * num_kb / p.split);
+    w.kb1 = static_cast<int>(static_cast<int64_t>(w.slice + 1) * num_kb / p.split);
+  } else {
+    w.tail = -1;
+    w.slice = 0;
+    t = unit + (has_tail ? k - 1 : k) * num_units;
+    w.kb0 = 0;
+    w.kb1 = num_kb;
+  }
+  tile_coords(t, num_m, num_n, p.raster_group, w.mb, w.nb);
+  return w;
+}
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int group, int &mb,
                                             int &nb) {
@@ -77,70 +132,80 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int gro
   nb = r / gm;
 }
 
-template <bool OUT_F16, bool BIAS_RELU>
-__device__ __forceinline__ void store_chunk(const GemmParams &p, int row, int col0,
-                                            const uint32_t (&r)[32]) {
-  float v[32];
+// Adds bias[col0 + j] (j < 32) to v and applies the ReLU.  Bias entries at
+// columns >= N are not read (those outputs are clipped by the store).
+__device__ __forceinline__ void bias_relu_32(const __half *__restrict__ bias, int col0, int N,
+                                             float (&v)[32]) {
+  if (col0 + 32 <= N) {
+    const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-  const bool full = col0 + 32 <= p.N;
-  if constexpr (BIAS_RELU) {
-    if (full) {
-      const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + col0);
+    for (int q = 0; q < 4; ++q) {
+      const uint4 w = __ldg(bp + q);
+      const __half2 *h = reinterpret_cast<const __half2 *>(&w);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 w = __ldg(bp + q);
-        const __half2 *h = reinterpret_cast<const __half2 *>(&w);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(h[e]);
-          v[q * 8 + 2 * e] += f.x;
-          v[q * 8 + 2 * e + 1] += f.y;
-        }
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        v[q * 8 + 2 * e] += f.x;
+        v[q * 8 + 2 * e + 1] += f.y;
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (col0 + j < p.N) v[j] += __half2float(p.bias[col0 + j]);
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
-  }
-  if constexpr (OUT_F16) {
-    __half *crow = reinterpret_cast<__half *>(p.C) + static_cast<int64_t>(row) * p.ldc + col0;
-    if (full) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 w;
-        __half2 *h = reinterpret_cast<__half2 *>(&w);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
-        reinterpret_cast<uint4 *>(crow)[q] = w;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (col0 + j < p.N) crow[j] = __float2half_rn(v[j]);
     }
   } else {
-    float *crow = reinterpret_cast<float *>(p.C) + static_cast<int64_t>(row) * p.ldc + col0;
-    if (full) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        reinterpret_cast<float4 *>(crow)[q] =
-            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    } else {
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < N) v[j] += __half2float(bias[col0 + j]);
+  }
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (col0 + j < p.N) crow[j] = v[j];
-    }
+  for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Writes one 128-byte row piece (eight 16-byte pieces) of a 32-row output box
+// in the TMA 128-byte swizzle: piece c of row r sits at (c ^ (r % 8)) * 16.
+__device__ __forceinline__ void st_box_row(uint32_t box, int r, const uint32_t (&w)[32],
+                                           int first_word) {
+  const uint32_t row = box + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t addr = row + static_cast<uint32_t>((c ^ (r & 7)) * 16);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                 "r"(w[first_word + 4 * c]), "r"(w[first_word + 4 * c + 1]),
+                 "r"(w[first_word + 4 * c + 2]), "r"(w[first_word + 4 * c + 3])
+                 : "memory");
+  }
+}
+
+// Plain predicated stores of one thread's row piece of 128 bytes (`w`, in
+// the output format: 32 fp32 words, or 64 fp16 values packed in pairs)
+// starting at column col0, only the columns below N.  Used for
+// the last column box when N * sizeof(out) is not a multiple of 16 bytes: the
+// TMA store's clipping would then write whole 16-byte pieces past column N.
+template <bool OUT_F16>
+__device__ __forceinline__ void store_row_tail(const GemmParams &p, int row, int col0,
+                                               const uint32_t (&w)[32]) {
+  if (row >= p.M) return;
+  if constexpr (OUT_F16) {
+    __half *c = reinterpret_cast<__half *>(p.C) + static_cast<int64_t>(row) * p.ldc + col0;
+#pragma unroll
+    for (int j = 0; j < 64; ++j)
+      if (col0 + j < p.N)
+        c[j] = __ushort_as_half(static_cast<unsigned short>(w[j / 2] >> (16 * (j & 1))));
+  } else {
+    float *c = reinterpret_cast<float *>(p.C) + static_cast<int64_t>(row) * p.ldc + col0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < p.N) c[j] = __uint_as_float(w[j]);
   }
 }
 
 template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
-                      const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using Plan = SmemPlan<CG, BN, STAGES>;
   constexpr int kTileM = kBM * CG;
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
@@ -170,8 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int num_m = (p.M + kTileM - 1) / kTileM;
   const int num_n = (p.N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
   const int num_kb = (p.K + kBK - 1) / kBK;
+  const int n_work = work_count(p, unit, num_units);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -180,13 +245,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4 * CG);  // one arrive per epilogue warp of each CTA
+      mbar_init(tempty_bar(a), kEpiWarps * CG);  // one arrive per epilogue warp of each CTA
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc<CG>(smem_u32(tmem_holder), Plan::kTmemCols);
@@ -207,12 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_parity = 0;
     bool ok = true;
-    for (int t = unit; t < num_tiles && ok; t += num_units) {
-      int mb, nb;
-      tile_coords(t, num_m, num_n, p.raster_group, mb, nb);
-      const int a_row = mb * kTileM + static_cast<int>(rank) * kBM;
-      const int b_col = nb * BN + static_cast<int>(rank) * Plan::kBNc;
-      for (int kb = 0; kb < num_kb; ++kb) {
+    for (int k = 0; k < n_work && ok; ++k) {
+      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+      const int a_row = w.mb * kTileM + static_cast<int>(rank) * kBM;
+      const int b_col = w.nb * BN + static_cast<int>(rank) * Plan::kBNc;
+      for (int kb = w.kb0; kb < w.kb1; ++kb) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
                        &g_device_error)) {
           ok = false;
@@ -273,7 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = unit; t < num_tiles && ok; t += num_units) {
+    for (int k = 0; k < n_work && ok; ++k) {
+      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
       if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
                      &g_device_error)) {
         ok = false;
@@ -281,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = w.kb0; kb < w.kb1; ++kb) {
         if (!mbar_wait(full_bar(stage), phase, abort_flag, p.limit_ns, kRoleMma,
                        &g_device_error)) {
           ok = false;
@@ -294,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(b0 + kk * 16 * 128, 8192, 1024);
-          mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (kb > w.kb0 || kk > 0) ? 1u : 0u);
         }
         mma_commit<CG>(empty_bar(stage));
         if (++stage == STAGES) {
@@ -314,40 +380,170 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue (every CTA)
-    const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ...
-    const int row_in_tile = static_cast<int>(rank) * kBM + quarter * 32 + lane;
+    // Warp w drains TMEM lanes 32*(w%4) .. +31 (the lanes a warp may access),
+    // 64 accumulator columns at a time, into two 4 KB boxes it owns in turn.
+    const int quarter = warp & 3;
+    const int box_row0_in_tile = static_cast<int>(rank) * kBM + quarter * 32;
+    const uint32_t box0 = smem_u32(smem + Plan::kOutOffset) +
+                          static_cast<uint32_t>((warp - 2) * 2) * kStageOutBytes;
     const uint32_t release_bar0 = (CG == 2) ? mapa_shared(tempty_bar(0), 0) : tempty_bar(0);
+    constexpr int kOutEsz = OUT_F16 ? 2 : 4;
+    constexpr int kBoxCols = 128 / kOutEsz;  // 64 fp16 or 32 fp32 columns per box
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = unit; t < num_tiles; t += num_units) {
-      int mb, nb;
-      tile_coords(t, num_m, num_n, p.raster_group, mb, nb);
+    uint32_t boxes_used = 0;
+
+    // Bias, ReLU, output rounding and the store of one 32-row x 64-column
+    // piece (this lane's row, columns col0 .. col0+63).
+    auto emit64 = [&](float (&va)[32], float (&vb)[32], int box_row0, int col0) {
+      if constexpr (BIAS_RELU) {
+        bias_relu_32(p.bias, col0, p.N, va);
+        bias_relu_32(p.bias, col0 + 32, p.N, vb);
+      }
+      if constexpr (OUT_F16) {
+        uint32_t h[32];  // 64 fp16 values, round to nearest even
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          h[j] = pack_half2(va[2 * j], va[2 * j + 1]);
+          h[16 + j] = pack_half2(vb[2 * j], vb[2 * j + 1]);
+        }
+        if (!p.n_aligned && col0 + kBoxCols > p.N) {
+          store_row_tail<true>(p, box_row0 + lane, col0, h);
+          return;
+        }
+        const uint32_t box = box0 + (boxes_used & 1u) * kStageOutBytes;
+        if (lane == 0) bulk_wait_group_read<1>();  // this box's previous store has read it
+        __syncwarp();
+        st_box_row(box, lane, h, 0);
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmC, box, col0, box_row0);
+          bulk_commit_group();
+        }
+        ++boxes_used;
+      } else {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (col0 + half * kBoxCols >= p.N) break;
+          uint32_t w[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(half == 0 ? va[j] : vb[j]);
+          if (!p.n_aligned && col0 + half * kBoxCols + kBoxCols > p.N) {
+            store_row_tail<false>(p, box_row0 + lane, col0 + half * kBoxCols, w);
+            continue;
+          }
+          const uint32_t box = box0 + (boxes_used & 1u) * kStageOutBytes;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          st_box_row(box, lane, w, 0);
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, box, col0 + half * kBoxCols, box_row0);
+            bulk_commit_group();
+          }
+          ++boxes_used;
+        }
+      }
+    };
+
+    for (int k = 0; k < n_work; ++k) {
+      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.limit_ns, kRoleEpilogue,
                      &g_device_error))
         break;
       tc_fence_after_sync();
-      const int row = mb * kTileM + row_in_tile;
+      const int box_row0 = w.mb * kTileM + box_row0_in_tile;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      // A k-slice of a tail tile writes its fp32 partial (this warp's 32 rows x
+      // BN columns, column by column so each store is 128 contiguous bytes).
+      float *part = nullptr;
+      if (w.tail >= 0)
+        part = p.ws + static_cast<int64_t>(((w.tail * p.split + w.slice) * CG + static_cast<int>(rank)) * 4 +
+                                           quarter) * (32 * BN);
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t r[32];
+      for (int ch = 0; ch < BN; ch += 64) {
+        uint32_t ra[32], rb[32];
         __syncwarp();
-        tmem_load_32cols(tbase + ch * 32, r);
-        const int col0 = nb * BN + ch * 32;
-        if (row < p.M && col0 < p.N) store_chunk<OUT_F16, BIAS_RELU>(p, row, col0, r);
+        tmem_load_2x32cols(tbase + ch, ra, rb);
+        if (ch + 64 >= BN) {
+          // Last read of this accumulator: hand it back to the MMA warp now,
+          // before the stores, so the next tile's main loop can start.
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (CG == 2)
+              mbar_arrive_cluster(release_bar0 + 8u * acc);
+            else
+              mbar_arrive(release_bar0 + 8u * acc);
+          }
+        }
+        if (part != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            st_global_cg(part + (ch + j) * 32 + lane, __uint_as_float(ra[j]));
+            st_global_cg(part + (ch + 32 + j) * 32 + lane, __uint_as_float(rb[j]));
+          }
+          continue;
+        }
+        const int col0 = w.nb * BN + ch;
+        if (box_row0 >= p.M || col0 >= p.N) continue;  // the whole 32 x 64 piece is clipped
+        float va[32], vb[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          va[j] = __uint_as_float(ra[j]);
+          vb[j] = __uint_as_float(rb[j]);
+        }
+        emit64(va, vb, box_row0, col0);
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (CG == 2)
-          mbar_arrive_cluster(release_bar0 + 8u * acc);
-        else
-          mbar_arrive(release_bar0 + 8u * acc);
+      if (part != nullptr) {
+        // Count this slice in; the warp that completes the count sums every
+        // slice's partial in slice order (a fixed order: the result does not
+        // depend on which slice finished last) and stores the tile piece.
+        uint32_t *counter = p.counters + (w.tail * CG + static_cast<int>(rank)) * 4 + quarter;
+        __syncwarp();
+        uint32_t before = 0;
+        if (lane == 0) {
+          __threadfence();
+          before = atomicAdd(counter, 1u);
+        }
+        before = __shfl_sync(0xffffffffu, before, 0);
+        if (before == static_cast<uint32_t>(p.split - 1)) {
+          __threadfence();
+          const float *part0 = p.ws + static_cast<int64_t>(((w.tail * p.split) * CG + static_cast<int>(rank)) * 4 +
+                                                           quarter) * (32 * BN);
+          const int64_t slice_stride = static_cast<int64_t>(CG) * 4 * 32 * BN;
+#pragma unroll 1
+          for (int ch = 0; ch < BN; ch += 64) {
+            const int col0 = w.nb * BN + ch;
+            if (box_row0 >= p.M || col0 >= p.N) continue;
+            float va[32], vb[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              va[j] = ld_global_cg(part0 + (ch + j) * 32 + lane);
+              vb[j] = ld_global_cg(part0 + (ch + 32 + j) * 32 + lane);
+            }
+            for (int sl = 1; sl < p.split; ++sl) {
+              const float *ps = part0 + sl * slice_stride;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                va[j] += ld_global_cg(ps + (ch + j) * 32 + lane);
+                vb[j] += ld_global_cg(ps + (ch + 32 + j) * 32 + lane);
+              }
+            }
+            emit64(va, vb, box_row0, col0);
+          }
+          __syncwarp();
+          if (lane == 0) atomicExch(counter, 0u);  // ready for the next call
+        }
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_group<0>();  // every store of this warp has completed
+    __syncwarp();
   }
 
   tc_fence_before_sync();
