@@ -46,10 +46,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FLUSH_BYTES = 256 << 20
 
 
+KERNEL_SOURCES = ("tlg_device.cuh", "tlg_gemm_kernel.cuh")  # device code of the GEMM kernel
+
+
 def kernel_source_hash() -> str:
+    """Hash of the GEMM kernel's device code: DRAM counters recorded for another hash are stale."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tiled_dense_gemm_tlg_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
@@ -176,26 +180,34 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def _reduce(x: float, world: int, op) -> float:
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time: the job is done when every rank is."""
+    import torch.distributed as dist
+
+    return _reduce(x, world, dist.ReduceOp.MAX if world > 1 else None)
 
 
 def sum_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(x, world, dist.ReduceOp.SUM if world > 1 else None)
+
+
+def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank's steps over the slowest rank's device time."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
 def cpu_oracle_rate(w: wl.Workload, target_s: float, threads: int, A=None, B=None, bias=None):
@@ -363,7 +375,7 @@ def main(argv=None):
 
     max_ms = max_over_ranks(gemm_ms, world)
     total_flops = w.flops * args.steps * world
-    value = total_flops / (max_ms * 1e-3) / 1e12
+    value = job_throughput(w.flops, args.steps, world, max_ms)
     ms_per_step = max_ms / args.steps
 
     # ---- end to end through the public API: pinned host inputs -> device -> GEMM -> pinned host output
