@@ -161,6 +161,42 @@ tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K,
                        void *stream);
 
 /*
+ * tlg_gemm_ex for callers that cannot allocate device memory.  (This entry
+ * point has no counterpart on the pages; it exists for library users.)
+ *
+ * Some callers cannot call cudaMalloc where they run a GEMM: a plugin inside
+ * a framework that owns all device memory through its own allocator, code
+ * with a fixed memory budget set at start-up, or a latency-critical path
+ * that must not risk the device-wide synchronisation an allocation can
+ * cause.  For them this call runs the split-K tail (config->split_k >= 2)
+ * with the library's own scratch: a static device array of 16 MiB that every
+ * GPU loading this library holds until the process exits.  Without
+ * config->split_k >= 2 no scratch is needed and the call is tlg_gemm_ex with
+ * no workspace.
+ *
+ * - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ * - The first call on each device looks up the array's device address (with
+ *   that device current) and may load the library's device code; make that
+ *   first call before any stream capture.
+ * - A schedule needing more than 16 MiB of scratch gives TLG_ERR_UNSUPPORTED
+ *   before anything is launched (tlg_gemm_workspace_size reports the need).
+ * - Every call on a device shares the one array, which keeps what the last
+ *   call left; each call clears the counters it needs on its stream first.
+ *   Calls that overlap on the GPU (different streams, or different host
+ *   threads without ordering) race on the array and give wrong results:
+ *   order them on one stream.
+ * - Arguments, layout, ownership and the other errors are as tlg_gemm_ex.
+ */
+tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K,
+                               const void *A, int64_t lda,
+                               const void *B, int64_t ldb,
+                               const void *bias,
+                               void *C, int64_t ldc,
+                               tlg_out out, tlg_epilogue epilogue,
+                               const tlg_config *config,
+                               void *stream);
+
+/*
  * Workspace bytes tlg_gemm_ex would use for this shape and configuration
  * (NULL = automatic) when given enough; 0 when every tile runs whole.
  * No kernel is launched; the only CUDA calls read device attributes.

@@ -42,7 +42,7 @@ TLG_OUT_F32, TLG_OUT_F16 = 0, 1
 TLG_EPI_NONE, TLG_EPI_BIAS_RELU = 0, 1
 
 EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-            "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
+            "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
             "tlg_version")
 
 
@@ -62,6 +62,8 @@ _lib.tlg_gemm_bias_relu_f16.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p
 _sz = ctypes.c_size_t
 _lib.tlg_gemm_ex.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i32, _i32,
                              ctypes.POINTER(tlg_config), _p, _sz, _p]
+_lib.tlg_gemm_ex_noalloc.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i32, _i32,
+                                     ctypes.POINTER(tlg_config), _p]
 _lib.tlg_gemm_workspace_size.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config),
                                          ctypes.POINTER(_sz)]
 _lib.tlg_choose_config.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config)]
@@ -71,7 +73,7 @@ _lib.tlg_status_string.argtypes = [_i32]
 _lib.tlg_status_string.restype = ctypes.c_char_p
 _lib.tlg_version.restype = ctypes.c_int32
 for _name in ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-              "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
+              "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
     getattr(_lib, _name).restype = _i32
 
 
@@ -186,6 +188,25 @@ def tlg_gemm_ex(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None = No
     _check(_lib.tlg_gemm_ex(M, N, K, pa, lda, pb, ldb, bias.data_ptr() if bias is not None else None,
                             pc, ldc, o, epi, ctypes.byref(cfg) if cfg is not None else None,
                             ws_ptr, ws_bytes, _stream_handle(stream, A, B, C)), "tlg_gemm_ex")
+    return C
+
+
+def tlg_gemm_ex_noalloc(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None = None,
+                        C: torch.Tensor | None = None, out: str = "f32", config: dict | None = None,
+                        stream=None):
+    """tlg_gemm_ex with the library's static scratch instead of a workspace (see tlg.h).
+    Allocates nothing in the library; C is allocated here only when not given."""
+    M, N, K = _shapes(A, B)
+    o = TLG_OUT_F32 if out == "f32" else TLG_OUT_F16
+    C = _out(C, M, N, torch.float32 if o == TLG_OUT_F32 else torch.float16, A)
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    pc, ldc = _mat(C, "C")
+    cfg = tlg_config(**{k: int(v) for k, v in config.items()}) if config is not None else None
+    epi = TLG_EPI_BIAS_RELU if bias is not None else TLG_EPI_NONE
+    _check(_lib.tlg_gemm_ex_noalloc(M, N, K, pa, lda, pb, ldb, bias.data_ptr() if bias is not None else None,
+                                    pc, ldc, o, epi, ctypes.byref(cfg) if cfg is not None else None,
+                                    _stream_handle(stream, A, B, C)), "tlg_gemm_ex_noalloc")
     return C
 
 

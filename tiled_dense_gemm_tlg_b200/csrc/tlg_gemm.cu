@@ -455,6 +455,46 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
   return fns_for(rv.idx, f16, br).launch(rv.sched.units, tmA, tmB, tmC, p, s);
 }
 
+// ---------------------------------------------------------------- allocation-free scratch
+//
+// Scratch for tlg_gemm_ex_noalloc: the split-K tail's partial sums and
+// counters live in this array instead of a caller workspace.  It is part of
+// the library's device image, so every GPU that loads the library holds its
+// 16 MiB until the process exits; no call allocates anything.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+struct StaticScratch {
+  bool ready = false;
+  void *ptr = nullptr;
+};
+StaticScratch g_static_scratch_of[kMaxDevices];
+
+// Device address of g_static_scratch on the current device.  The host-side
+// name is only a stand-in for the symbol; the address a kernel may use comes
+// from cudaGetSymbolAddress, asked once per device with that device current.
+tlg_status static_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return TLG_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return TLG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  StaticScratch &s = g_static_scratch_of[dev];
+  if (!s.ready) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return TLG_ERR_CUDA;
+    }
+    s.ptr = p;
+    s.ready = true;
+  }
+  *out = s.ptr;
+  return TLG_OK;
+}
+
 tlg_status resolve_public(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_epilogue epilogue,
                           const tlg_config *req, size_t ws_bytes, Resolved *rv) {
   if (out != TLG_OUT_F32 && out != TLG_OUT_F16) return TLG_ERR_INVALID_ARG;
@@ -499,6 +539,34 @@ tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K, const void *A, int64_t l
                        size_t workspace_bytes, void *stream) {
   return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, workspace,
                    workspace_bytes, stream);
+}
+
+tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
+                               const void *B, int64_t ldb, const void *bias, void *C, int64_t ldc,
+                               tlg_out out, tlg_epilogue epilogue, const tlg_config *config,
+                               void *stream) {
+  const bool split = config != nullptr && config->split_k >= 2;
+  if (!split)  // no scratch needed: exactly tlg_gemm_ex without a workspace
+    return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, nullptr, 0,
+                     stream);
+  // Reject a schedule whose scratch would not fit before touching anything.
+  if (M > 0 && N > 0 && K > 0) {
+    Resolved rv;
+    const tlg_status rs = resolve_public(M, N, K, out, epilogue, config, SIZE_MAX, &rv);
+    if (rs != TLG_OK) return rs;
+    if (rv.sched.workspace > kStaticScratchBytes) return TLG_ERR_UNSUPPORTED;
+  }
+  void *scratch = nullptr;
+  const tlg_status ss = static_scratch(&scratch);
+  if (ss != TLG_OK) return ss;
+  // The counters must start at zero; the array keeps whatever the last call left.
+  if (M > 0 && N > 0 && K > 0 &&
+      cudaMemsetAsync(scratch, 0, kCounterBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return TLG_ERR_CUDA;
+  }
+  return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, scratch,
+                   kStaticScratchBytes, stream);
 }
 
 tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
