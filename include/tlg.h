@@ -107,7 +107,8 @@ typedef enum tlg_epilogue { TLG_EPI_NONE = 0, TLG_EPI_BIAS_RELU = 1 } tlg_epilog
  * Kernel configuration.  Zero in any field means "choose for me" (the
  * library's per-shape table, the analogue of the pages' cached tuned
  * configurations: "tilelang operator-compilation walkthrough" section 5.3).
- *   block_n     : output tile width, 64, 128 or 256 columns
+ *   block_n     : output tile width, 64, 128 or 256 columns, or 512 for a CTA
+ *                 pair whose tile fills TMEM with two 256-column halves
  *   stages      : depth of the shared-memory operand ring (fixed per tile shape)
  *   cta_group   : 1 (one SM per 128-row tile) or 2 (an SM pair per 256-row tile)
  *   raster_group: number of tile rows walked together for L2 reuse, 1..64

@@ -19,7 +19,7 @@ SIZES = [1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 256, 257]
 OUTS = [("f32", False), ("f16", False), ("f16", True)]
 WIDTHS = [64, 128, 256]
 # every kernel variant the library builds: (CTAs per tile, tile width, ring stages)
-TILES = [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6)]
+TILES = [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6), (2, 512, 4)]
 
 
 def tile_cfg(tile):
@@ -72,7 +72,7 @@ def test_every_tile_on_multi_tile_ragged_shape(lib, tile, out, bias_relu):
     assert ok, f"worst err/bound {worst:.3g} at {idx}"
 
 
-@pytest.mark.parametrize("tile", [(1, 128, 6), (2, 256, 6)])
+@pytest.mark.parametrize("tile", [(1, 128, 6), (2, 256, 6), (2, 512, 4)])
 @pytest.mark.parametrize("raster_group,max_ctas", [(1, 0), (3, 0), (64, 0), (8, 2), (8, 7)])
 def test_scheduler_variants(lib, tile, raster_group, max_ctas):
     # fewer CTAs than tiles makes each CTA loop over many tiles and both TMEM accumulators

@@ -102,7 +102,7 @@ def test_integer_inputs_are_bit_exact(tlg, name):
         assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), want)
 
 
-@pytest.mark.parametrize("tile", [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6)])
+@pytest.mark.parametrize("tile", [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6), (2, 512, 4)])
 def test_every_tile_on_the_bias_relu_workload(tlg, tile):
     # the full-size bias+ReLU workload under each kernel variant the library builds
     w = wl.WORKLOADS["gemm_bias_relu_4096_f16"]

@@ -12,7 +12,7 @@ from gpu_util import gemm_padded
 
 pytestmark = pytest.mark.gpu
 
-TILES = [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6)]
+TILES = [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6), (2, 512, 4)]
 OUTS = [("f32", False), ("f16", False), ("f16", True)]
 
 

@@ -92,9 +92,10 @@ bool overlaps(uintptr_t a0, uintptr_t a1, uintptr_t b0, uintptr_t b1) { return a
 
 struct KernelCfg {
   int cta_group;
-  int block_n;
+  int block_n;  // tile width; 512 = two 256-column MMA halves filling TMEM
   int stages;
-  double eff;  // fraction of the MMA peak one tile sustains (used to rank tile shapes)
+  double eff;         // sustained fraction of the MMA peak, relative (ranks tile shapes)
+  double exposed_kb;  // k-blocks per tile the main loop waits for the epilogue
 };
 
 // Kernel variants the library is built with.  A tile is 128*cta_group rows by
@@ -103,8 +104,11 @@ struct KernelCfg {
 // 227 KB of shared memory next to 32 KB of output staging.
 // `eff` is measured: TFLOP/s of each shape on a B200 at M = N = K = 4096 and
 // 8192 after dividing out the wave count, relative to the 2 x 256 pair tile.
-constexpr KernelCfg kBuilt[] = {
-    {1, 64, 8, 0.35}, {1, 128, 6, 0.60}, {1, 256, 4, 0.90}, {2, 128, 8, 0.60}, {2, 256, 6, 1.00}};
+// The 512-wide tile moves 25 % fewer operand bytes per FLOP, which under the
+// 1000 W cap buys a higher clock (sustained at 8192^3: 1297 vs 1170 MHz), but
+// its single accumulator leaves part of each epilogue exposed (exposed_kb).
+constexpr KernelCfg kBuilt[] = {{1, 64, 8, 0.35, 0},  {1, 128, 6, 0.60, 0}, {1, 256, 4, 0.90, 0},
+                                {2, 128, 8, 0.60, 0}, {2, 256, 6, 1.00, 0}, {2, 512, 4, 1.07, 8}};
 constexpr int kNumBuilt = sizeof(kBuilt) / sizeof(kBuilt[0]);
 
 // Per device and instantiation: kernel attributes set, co-resident work units.
@@ -113,9 +117,11 @@ struct LaunchState {
   int units = 0;
 };
 
-template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
+template <int CG, int TN, int STAGES, bool OUT_F16, bool BIAS_RELU>
 struct Variant {
-  using Plan = SmemPlan<CG, BN, STAGES>;
+  static constexpr int NH = TN > 256 ? 2 : 1;  // MMA halves per tile
+  static constexpr int BN = TN / NH;           // the MMA's N
+  using Plan = SmemPlan<CG, BN, STAGES, NH>;
 
   static void fill_launch(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, cudaStream_t s) {
     *cfg = {};
@@ -136,7 +142,7 @@ struct Variant {
   // or the number of 2-CTA clusters the occupancy calculator admits.
   static tlg_status units(int dev, int sms, int *out) {
     static LaunchState state[kMaxDevices];
-    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU>;
+    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH>;
     std::lock_guard<std::mutex> lock(g_mutex);
     LaunchState &st = state[dev];
     if (!st.ready) {
@@ -170,7 +176,7 @@ struct Variant {
     fill_launch(&cfg, attr, s);
     cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU>, tmA, tmB, tmC, p);
+        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH>, tmA, tmB, tmC, p);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return TLG_ERR_CUDA;
@@ -191,9 +197,9 @@ struct VariantFns {
   { TLG_FNS(CG, BN, ST, false, false), TLG_FNS(CG, BN, ST, true, false), TLG_FNS(CG, BN, ST, true, true) }
 
 // [variant, same order as kBuilt][f32 | f16 | f16 bias+ReLU]
-const VariantFns kVariantFns[kNumBuilt][3] = {TLG_VARIANT(1, 64, 8), TLG_VARIANT(1, 128, 6),
-                                              TLG_VARIANT(1, 256, 4), TLG_VARIANT(2, 128, 8),
-                                              TLG_VARIANT(2, 256, 6)};
+const VariantFns kVariantFns[kNumBuilt][3] = {TLG_VARIANT(1, 64, 8),  TLG_VARIANT(1, 128, 6),
+                                              TLG_VARIANT(1, 256, 4),  TLG_VARIANT(2, 128, 8),
+                                              TLG_VARIANT(2, 256, 6),  TLG_VARIANT(2, 512, 4)};
 #undef TLG_VARIANT
 #undef TLG_FNS
 
@@ -290,7 +296,9 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
     (void)ws_bytes;
     if (!plan(tiles, resident, num_kb, r.split_k == 0 ? 1 : r.split_k, k.cta_group, k.block_n, &sch))
       continue;
-    const double cost = sch.cost * static_cast<double>(tile_m * k.block_n) / (k.cta_group * k.eff);
+    const double per_unit_tiles = static_cast<double>(tiles + sch.units - 1) / sch.units;
+    const double cost = (sch.cost + per_unit_tiles * k.exposed_kb) *
+                        static_cast<double>(tile_m * k.block_n) / (k.cta_group * k.eff);
     if (!found || cost < best_cost * 0.999) {
       found = true;
       best_cost = cost;

@@ -41,13 +41,16 @@ constexpr uint32_t kStageOutBytes = 32 * 128;   // one TMA store box: 32 rows x 
 __device__ uint32_t g_device_error;
 
 // Shared-memory plan of one CTA.  CG CTAs (1 or 2) compute one tile of
-// 128*CG rows by BN columns; each CTA stages its own 128 rows of A and its own
-// BN/CG columns of B per k-block, plus two 4 KB output boxes per epilogue warp.
-template <int CG, int BN, int STAGES>
+// 128*CG rows by NH*BN columns (BN = the MMA's N; NH = 1, or 2 for a tile of
+// two MMA halves that fills TMEM); each CTA stages its own 128 rows of A and
+// its own BN/CG columns of each half of B per k-block, plus two 4 KB output
+// boxes per epilogue warp.
+template <int CG, int BN, int STAGES, int NH = 1>
 struct SmemPlan {
-  static constexpr int kBNc = BN / CG;  // B columns held by one CTA
+  static constexpr int kBNc = BN / CG;  // B columns of one MMA half held by one CTA
   static constexpr uint32_t kABytes = kBM * kBK * 2;
-  static constexpr uint32_t kBBytes = kBK * kBNc * 2;
+  static constexpr uint32_t kHalfBBytes = kBK * kBNc * 2;
+  static constexpr uint32_t kBBytes = kHalfBBytes * NH;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kOutOffset = STAGES * kStageBytes;
   static constexpr uint32_t kOutBytes = kEpiWarps * 2 * kStageOutBytes;
@@ -201,14 +204,21 @@ __device__ __forceinline__ void store_row_tail(const GemmParams &p, int row, int
   }
 }
 
-template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU>
+// NH == 1: each tile is one BN-wide accumulator and two accumulators
+// alternate in TMEM, so the epilogue of one tile overlaps the next tile's
+// main loop.  NH == 2: each tile is 2*BN wide and fills TMEM with two
+// BN-column halves; the epilogue hands half 0 back before draining half 1, so
+// the next tile's MMAs into half 0 start while half 1 is still being stored.
+template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU, int NH = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
-  using Plan = SmemPlan<CG, BN, STAGES>;
+  using Plan = SmemPlan<CG, BN, STAGES, NH>;
   constexpr int kTileM = kBM * CG;
+  constexpr int kTileN = BN * NH;
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
+  static_assert(NH == 1 || NH == 2, "one accumulator per tile, or two halves");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
 
   extern __shared__ uint8_t smem_raw[];
@@ -234,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_units = (CG == 2) ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
   const bool leader = rank == 0;
   const int num_m = (p.M + kTileM - 1) / kTileM;
-  const int num_n = (p.N + BN - 1) / BN;
+  const int num_n = (p.N + kTileN - 1) / kTileN;
   const int num_kb = (p.K + kBK - 1) / kBK;
   const int n_work = work_count(p, unit, num_units);
 
@@ -276,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < n_work && ok; ++k) {
       const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
       const int a_row = w.mb * kTileM + static_cast<int>(rank) * kBM;
-      const int b_col = w.nb * BN + static_cast<int>(rank) * Plan::kBNc;
+      const int b_col = w.nb * kTileN + static_cast<int>(rank) * Plan::kBNc;
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
                        &g_device_error)) {
@@ -289,16 +299,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(full_bar(stage), Plan::kStageBytes);
           tma_load_2d(a_dst, &tmA, full_bar(stage), kb * kBK, a_row);
 #pragma unroll
-          for (int c = 0; c < Plan::kBNc / 64; ++c)
-            tma_load_2d(b_dst + c * 8192, &tmB, full_bar(stage), b_col + c * 64, kb * kBK);
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int c = 0; c < Plan::kBNc / 64; ++c)
+              tma_load_2d(b_dst + h * Plan::kHalfBBytes + c * 8192, &tmB, full_bar(stage),
+                          b_col + h * BN + c * 64, kb * kBK);
         } else {
           // The leader's full barrier counts the bytes of both CTAs' loads.
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * Plan::kStageBytes);
           const uint32_t bar = mapa_shared(full_bar(stage), 0);
           tma_load_2d_pair(a_dst, &tmA, bar, kb * kBK, a_row);
 #pragma unroll
-          for (int c = 0; c < Plan::kBNc / 64; ++c)
-            tma_load_2d_pair(b_dst + c * 8192, &tmB, bar, b_col + c * 64, kb * kBK);
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int c = 0; c < Plan::kBNc / 64; ++c)
+              tma_load_2d_pair(b_dst + h * Plan::kHalfBBytes + c * 8192, &tmB, bar,
+                               b_col + h * BN + c * 64, kb * kBK);
         }
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -335,6 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc = make_idesc_f16(kTileM, BN);
     int stage = 0;
     uint32_t phase = 0;
+    // Accumulator slots are the two BN-column halves of TMEM.  NH == 1: tiles
+    // alternate between them (acc); NH == 2: every tile uses both.
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -346,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      bool half1_free = NH == 1;  // NH == 2: waited for just before its first MMA
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
         if (!mbar_wait(full_bar(stage), phase, abort_flag, p.limit_ns, kRoleMma,
                        &g_device_error)) {
@@ -357,11 +375,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a0 = smem_u32(sA + stage * Plan::kABytes);
         const uint32_t b0 = smem_u32(sB + stage * Plan::kBBytes);
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(b0 + kk * 16 * 128, 8192, 1024);
-          mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (kb > w.kb0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < NH; ++h) {
+          if (NH == 2 && h == 1 && !half1_free) {
+            if (!mbar_wait(tempty_bar(1), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
+                           &g_device_error)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            half1_free = true;
+          }
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((NH == 1 ? acc : h) * BN);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bdesc =
+                smem_desc_sw128(b0 + h * Plan::kHalfBBytes + kk * 16 * 128, 8192, 1024);
+            mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (kb > w.kb0 || kk > 0) ? 1u : 0u);
+          }
         }
+        if (!ok) break;
         mma_commit<CG>(empty_bar(stage));
         if (++stage == STAGES) {
           stage = 0;
@@ -370,8 +403,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       mma_commit<CG>(tfull_bar(acc));
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (NH == 1) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;  // both halves' barriers complete once per tile
+      }
     }
     if (!ok) {
       // Wait for the MMAs already in flight before TMEM and shared memory are released.
@@ -455,40 +492,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       tc_fence_after_sync();
       const int box_row0 = w.mb * kTileM + box_row0_in_tile;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
       // A k-slice of a tail tile writes its fp32 partial (this warp's 32 rows x
-      // BN columns, column by column so each store is 128 contiguous bytes).
+      // kTileN columns, column by column so each store is 128 contiguous bytes).
       float *part = nullptr;
       if (w.tail >= 0)
         part = p.ws + static_cast<int64_t>(((w.tail * p.split + w.slice) * CG + static_cast<int>(rank)) * 4 +
-                                           quarter) * (32 * BN);
+                                           quarter) * (32 * kTileN);
 #pragma unroll 1
-      for (int ch = 0; ch < BN; ch += 64) {
+      for (int tc = 0; tc < kTileN; tc += 64) {
+        const int slot = NH == 1 ? acc : tc / BN;  // TMEM half holding these columns
+        const int ch = tc % BN;
         uint32_t ra[32], rb[32];
         __syncwarp();
-        tmem_load_2x32cols(tbase + ch, ra, rb);
+        tmem_load_2x32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(slot * BN + ch),
+                           ra, rb);
         if (ch + 64 >= BN) {
-          // Last read of this accumulator: hand it back to the MMA warp now,
-          // before the stores, so the next tile's main loop can start.
+          // Last read of this accumulator half: hand it back to the MMA warp
+          // now, before the stores, so the next tile's main loop can start.
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) {
             if constexpr (CG == 2)
-              mbar_arrive_cluster(release_bar0 + 8u * acc);
+              mbar_arrive_cluster(release_bar0 + 8u * slot);
             else
-              mbar_arrive(release_bar0 + 8u * acc);
+              mbar_arrive(release_bar0 + 8u * slot);
           }
         }
         if (part != nullptr) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            st_global_cg(part + (ch + j) * 32 + lane, __uint_as_float(ra[j]));
-            st_global_cg(part + (ch + 32 + j) * 32 + lane, __uint_as_float(rb[j]));
+            st_global_cg(part + (tc + j) * 32 + lane, __uint_as_float(ra[j]));
+            st_global_cg(part + (tc + 32 + j) * 32 + lane, __uint_as_float(rb[j]));
           }
           continue;
         }
-        const int col0 = w.nb * BN + ch;
+        const int col0 = w.nb * kTileN + tc;
         if (box_row0 >= p.M || col0 >= p.N) continue;  // the whole 32 x 64 piece is clipped
         float va[32], vb[32];
 #pragma unroll
@@ -513,11 +552,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (before == static_cast<uint32_t>(p.split - 1)) {
           __threadfence();
           const float *part0 = p.ws + static_cast<int64_t>(((w.tail * p.split) * CG + static_cast<int>(rank)) * 4 +
-                                                           quarter) * (32 * BN);
-          const int64_t slice_stride = static_cast<int64_t>(CG) * 4 * 32 * BN;
+                                                           quarter) * (32 * kTileN);
+          const int64_t slice_stride = static_cast<int64_t>(CG) * 4 * 32 * kTileN;
 #pragma unroll 1
-          for (int ch = 0; ch < BN; ch += 64) {
-            const int col0 = w.nb * BN + ch;
+          for (int ch = 0; ch < kTileN; ch += 64) {
+            const int col0 = w.nb * kTileN + ch;
             if (box_row0 >= p.M || col0 >= p.N) continue;
             float va[32], vb[32];
 #pragma unroll
@@ -539,8 +578,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) atomicExch(counter, 0u);  // ready for the next call
         }
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (NH == 1) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
     }
     if (lane == 0) bulk_wait_group<0>();  // every store of this warp has completed
     __syncwarp();
