@@ -118,6 +118,11 @@ typedef enum tlg_epilogue { TLG_EPI_NONE = 0, TLG_EPI_BIAS_RELU = 1 } tlg_epilog
  *                 (needs a workspace).  The automatic choice does not split:
  *                 on a B200 under its power cap a split tail measured no
  *                 faster at 4096^3 and slower at 1024^3.
+ *   overlap_prev: 1 = the kernel may begin its set-up (barriers, TMEM, tensor
+ *                 maps) while the previous kernel in the stream is still
+ *                 finishing (programmatic dependent launch); it reads and
+ *                 writes global memory only after that kernel has completed.
+ *                 0 (default) = ordinary stream order.
  * A combination the library does not provide gives TLG_ERR_UNSUPPORTED.
  */
 typedef struct tlg_config {
@@ -127,6 +132,7 @@ typedef struct tlg_config {
     int32_t raster_group;
     int32_t max_ctas;
     int32_t split_k;
+    int32_t overlap_prev;
 } tlg_config;
 
 /*

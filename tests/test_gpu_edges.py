@@ -85,6 +85,27 @@ def test_scheduler_variants(lib, tile, raster_group, max_ctas):
     assert ok, f"worst err/bound {worst:.3g} at {idx}"
 
 
+@pytest.mark.parametrize("tile", [(1, 128, 6), (2, 256, 6), (2, 512, 4)])
+def test_dependent_launch_waits_for_the_previous_kernel(tlg, tile):
+    # GEMM 2 reads GEMM 1's output and is launched to overlap it.  Integer
+    # operands keep every value exact, so GEMM 2's expected result comes from
+    # the oracle alone: C1 = A1.B1 exactly (|C1| <= 4*K1 <= 2048, exact in fp16).
+    M, K1, N1, N2 = 1000, 256, 520, 392
+    A1, B1, _ = wl.integer_operands(M, N1, K1, lo=-2, hi=2, seed=14)
+    _, B2, _ = wl.integer_operands(1, N2, N1, lo=-1, hi=1, seed=15)
+    C1_ref = oracle.gemm(A1, B1)
+    assert np.abs(C1_ref).max() <= 2048
+    C2_ref = oracle.gemm(oracle.f16_encode_rne(C1_ref), B2)
+    cfg = {"cta_group": tile[0], "block_n": tile[1], "overlap_prev": 1}
+    dA1, dB1, dB2 = A1.cuda(), B1.cuda(), B2.cuda()
+    for _ in range(3):
+        C1 = torch.full((M, N1), float("nan"), dtype=torch.float16, device="cuda")
+        tlg.tlg_gemm_ex(dA1, dB1, C=C1, out="f16", config=cfg)
+        C2 = tlg.tlg_gemm_ex(C1, dB2, out="f32", config=cfg)
+        torch.cuda.synchronize()
+        assert np.array_equal(C2.double().cpu().numpy(), C2_ref)
+
+
 def test_transpose_identity_on_gpu(tlg):
     A, B, _ = wl.make_operands(304, 200, 136, "uniform", seed=8)  # every ld a multiple of 8
     C1 = tlg.tlg_gemm_f16f32(A.cuda(), B.cuda())

@@ -181,6 +181,21 @@ __device__ __forceinline__ float ld_global_cg(const float *ptr) {
   return v;
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Block until the grids this launch depends on (the previous kernel in the
+// stream, when launched with programmatic stream serialization) have
+// completed and their memory is visible; a no-op otherwise.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel in the stream, if it was launched as a programmatic
+// dependent, to begin its own prologue.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -123,19 +123,30 @@ struct Variant {
   static constexpr int BN = TN / NH;           // the MMA's N
   using Plan = SmemPlan<CG, BN, STAGES, NH>;
 
-  static void fill_launch(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, cudaStream_t s) {
+  // attr must hold 2 entries.  With overlap_prev the kernel may start while
+  // the previous kernel in the stream finishes (programmatic stream
+  // serialization); it waits for that kernel before touching global memory.
+  static void fill_launch(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, cudaStream_t s,
+                          bool overlap_prev = false) {
     *cfg = {};
     cfg->blockDim = dim3(kThreads, 1, 1);
     cfg->dynamicSmemBytes = Plan::kDynamicBytes;
     cfg->stream = s;
-    if (CG == 2) {
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 2;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg->attrs = attr;
-      cfg->numAttrs = 1;
+    int n = 0;
+    if (overlap_prev) {
+      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[n].val.programmaticStreamSerializationAllowed = 1;
+      ++n;
     }
+    if (CG == 2) {
+      attr[n].id = cudaLaunchAttributeClusterDimension;
+      attr[n].val.clusterDim.x = 2;
+      attr[n].val.clusterDim.y = 1;
+      attr[n].val.clusterDim.z = 1;
+      ++n;
+    }
+    cfg->attrs = attr;
+    cfg->numAttrs = n;
   }
 
   // Work units (CTAs, or CTA pairs) that can be resident at once: one per SM,
@@ -154,7 +165,7 @@ struct Variant {
       int n = sms;
       if (CG == 2) {
         cudaLaunchConfig_t cfg;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         fill_launch(&cfg, attr, nullptr);
         cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
         if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
@@ -170,10 +181,11 @@ struct Variant {
   }
 
   static tlg_status launch(int units, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                           const CUtensorMap &tmC, const GemmParams &p, cudaStream_t s) {
+                           const CUtensorMap &tmC, const GemmParams &p, bool overlap_prev,
+                           cudaStream_t s) {
     cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute attr[1];
-    fill_launch(&cfg, attr, s);
+    cudaLaunchAttribute attr[2];
+    fill_launch(&cfg, attr, s, overlap_prev);
     cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(
         &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH>, tmA, tmB, tmC, p);
@@ -188,7 +200,7 @@ struct Variant {
 struct VariantFns {
   tlg_status (*units)(int, int, int *);
   tlg_status (*launch)(int, const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                       const GemmParams &, cudaStream_t);
+                       const GemmParams &, bool, cudaStream_t);
 };
 
 #define TLG_FNS(CG, BN, ST, F16, BR) \
@@ -271,7 +283,8 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
   tlg_config r = {};
   if (req != nullptr) r = *req;
   if (r.raster_group < 0 || r.raster_group > 64 || r.max_ctas < 0 || r.split_k < 0 ||
-      r.split_k > 16 || r.stages < 0 || r.block_n < 0 || r.cta_group < 0)
+      r.split_k > 16 || r.stages < 0 || r.block_n < 0 || r.cta_group < 0 ||
+      (r.overlap_prev != 0 && r.overlap_prev != 1))
     return TLG_ERR_UNSUPPORTED;
   double best_cost = 0;
   bool found = false;
@@ -313,6 +326,7 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
   out->cfg.raster_group = r.raster_group != 0 ? r.raster_group : 8;
   out->cfg.max_ctas = r.max_ctas;
   out->cfg.split_k = out->sched.split;
+  out->cfg.overlap_prev = r.overlap_prev;
   return TLG_OK;
 }
 
@@ -460,7 +474,7 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
   p.counters = static_cast<uint32_t *>(ws);
   p.ws = ws != nullptr ? reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes)
                        : nullptr;
-  return fns_for(rv.idx, f16, br).launch(rv.sched.units, tmA, tmB, tmC, p, s);
+  return fns_for(rv.idx, f16, br).launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
 }
 
 // ---------------------------------------------------------------- allocation-free scratch

@@ -276,6 +276,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_holder);
+  // Everything above touched only this CTA's shared memory and TMEM, so it may
+  // overlap the previous kernel in the stream; global memory (A, B, bias, C,
+  // the workspace) is touched only after that kernel has completed.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- producer (every CTA)
