@@ -285,6 +285,8 @@ def main(argv=None):
     ap.add_argument("--config", default=None, help="JSON tlg_config override (tuning sweeps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layout", default="NN", choices=["NN", "NT", "TN", "TT"],
+                    help="op(A), op(B): T = that operand is stored transposed (tlg_gemm_op)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
@@ -300,6 +302,11 @@ def main(argv=None):
     dev = torch.device("cuda", local if world > 1 else 0)
     stream = torch.cuda.current_stream(dev)
     A, B, bias = wl.workload_operands(w, seed=rank)
+    at, bt = args.layout[0] == "T", args.layout[1] == "T"
+    if at:
+        A = A.t().contiguous()  # stored K x M; the product uses its transpose
+    if bt:
+        B = B.t().contiguous()  # stored N x K
     dA, dB = A.to(dev), B.to(dev)
     dbias = bias.to(dev) if bias is not None else None
     dC = torch.empty((w.M, w.N), dtype=torch.float32 if w.out == "f32" else torch.float16, device=dev)
@@ -311,8 +318,9 @@ def main(argv=None):
     ws = tlg.tlg_workspace(ws_bytes, device=dev) if ws_bytes > 0 else None
     plain_name = ("tlg_gemm_bias_relu_f16" if w.bias_relu else
                   ("tlg_gemm_f16f16" if w.out == "f16" else "tlg_gemm_f16f32"))
-    use_ex = ws is not None or override is not None
-    entry = "tlg_gemm_ex" if use_ex else plain_name
+    use_op = at or bt
+    use_ex = (ws is not None or override is not None) and not use_op
+    entry = "tlg_gemm_op" if use_op else ("tlg_gemm_ex" if use_ex else plain_name)
 
     def plain_step():
         if w.bias_relu:
@@ -323,7 +331,10 @@ def main(argv=None):
             tlg.tlg_gemm_f16f32(dA, dB, dC, stream=stream)
 
     def step():
-        if use_ex:
+        if use_op:
+            tlg.tlg_gemm_op(dA, dB, args.layout[0], args.layout[1], dbias, dC, out=w.out, config=override,
+                            workspace=ws, stream=stream)
+        elif use_ex:
             tlg.tlg_gemm_ex(dA, dB, dbias, dC, out=w.out, config=override, workspace=ws, stream=stream)
         else:
             plain_step()
@@ -362,7 +373,7 @@ def main(argv=None):
 
     # The same steps through the plain entry point (no workspace), for comparison.
     plain = None
-    if use_ex and override is None:
+    if use_ex and override is None and not use_op:
         for _ in range(args.warmup):
             flush.fill_(1.0)
             plain_step()
@@ -443,7 +454,8 @@ def main(argv=None):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": dict(workload_config(w, kcfg), entry_point=entry, workspace_bytes=ws_bytes),
+        "config": dict(workload_config(w, kcfg), entry_point=entry, workspace_bytes=ws_bytes,
+                       layout=args.layout),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "plain_entry_point": plain,
         "gpu_launches": args.steps,
         "clocks": clk,

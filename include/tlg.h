@@ -203,6 +203,32 @@ tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K,
                                const tlg_config *config,
                                void *stream);
 
+/* Whether an operand is used as stored (N) or transposed (T). */
+typedef enum tlg_op { TLG_OP_N = 0, TLG_OP_T = 1 } tlg_op;
+
+/*
+ * C = op(A) . op(B) with the same epilogues, configuration and workspace as
+ * tlg_gemm_ex, for operands stored transposed: the products of the pages'
+ * autograd wrapper, grad_A = grad_C . B^T and grad_B = A^T . grad_C ("TileLang
+ * Python DSL practice", codechina.net/.../126997, section 5.1).
+ *   op_a == TLG_OP_N: A is M x K row-major, lda >= K (as tlg_gemm_ex).
+ *   op_a == TLG_OP_T: A is stored K x M row-major, lda >= M; op(A) = A^T.
+ *   op_b == TLG_OP_N: B is K x N row-major, ldb >= N (as tlg_gemm_ex).
+ *   op_b == TLG_OP_T: B is stored N x K row-major, ldb >= K; op(B) = B^T.
+ * C is always M x N row-major.  The 16-byte alignment rules apply to the
+ * stored matrices (lda*2, ldb*2 multiples of 16).  Other arguments and errors
+ * as tlg_gemm_ex; an op other than N or T is TLG_ERR_INVALID_ARG.
+ */
+tlg_status tlg_gemm_op(int64_t M, int64_t N, int64_t K,
+                       tlg_op op_a, const void *A, int64_t lda,
+                       tlg_op op_b, const void *B, int64_t ldb,
+                       const void *bias,
+                       void *C, int64_t ldc,
+                       tlg_out out, tlg_epilogue epilogue,
+                       const tlg_config *config,
+                       void *workspace, size_t workspace_bytes,
+                       void *stream);
+
 /*
  * Workspace bytes tlg_gemm_ex would use for this shape and configuration
  * (NULL = automatic) when given enough; 0 when every tile runs whole.

@@ -40,9 +40,10 @@ _lib = ctypes.CDLL(LIB_PATH)
 TLG_OK, TLG_ERR_INVALID_ARG, TLG_ERR_ALIGNMENT, TLG_ERR_UNSUPPORTED, TLG_ERR_CUDA, TLG_ERR_TIMEOUT = range(6)
 TLG_OUT_F32, TLG_OUT_F16 = 0, 1
 TLG_EPI_NONE, TLG_EPI_BIAS_RELU = 0, 1
+TLG_OP_N, TLG_OP_T = 0, 1
 
 EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-            "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
+            "tlg_gemm_op", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
             "tlg_version")
 
 
@@ -62,6 +63,8 @@ _lib.tlg_gemm_bias_relu_f16.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p
 _sz = ctypes.c_size_t
 _lib.tlg_gemm_ex.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i32, _i32,
                              ctypes.POINTER(tlg_config), _p, _sz, _p]
+_lib.tlg_gemm_op.argtypes = [_i64, _i64, _i64, _i32, _p, _i64, _i32, _p, _i64, _p, _p, _i64, _i32, _i32,
+                             ctypes.POINTER(tlg_config), _p, _sz, _p]
 _lib.tlg_gemm_ex_noalloc.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i32, _i32,
                                      ctypes.POINTER(tlg_config), _p]
 _lib.tlg_gemm_workspace_size.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config),
@@ -73,7 +76,7 @@ _lib.tlg_status_string.argtypes = [_i32]
 _lib.tlg_status_string.restype = ctypes.c_char_p
 _lib.tlg_version.restype = ctypes.c_int32
 for _name in ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-              "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
+              "tlg_gemm_op", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
     getattr(_lib, _name).restype = _i32
 
 
@@ -188,6 +191,35 @@ def tlg_gemm_ex(A: torch.Tensor, B: torch.Tensor, bias: torch.Tensor | None = No
     _check(_lib.tlg_gemm_ex(M, N, K, pa, lda, pb, ldb, bias.data_ptr() if bias is not None else None,
                             pc, ldc, o, epi, ctypes.byref(cfg) if cfg is not None else None,
                             ws_ptr, ws_bytes, _stream_handle(stream, A, B, C)), "tlg_gemm_ex")
+    return C
+
+
+def tlg_gemm_op(A: torch.Tensor, B: torch.Tensor, op_a: str = "N", op_b: str = "N",
+                bias: torch.Tensor | None = None, C: torch.Tensor | None = None, out: str = "f32",
+                config: dict | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """C = op(A).op(B): ``op_a == "T"`` means A is stored K x M and its transpose is used;
+    ``op_b == "T"`` means B is stored N x K.  Stored matrices are row-major."""
+    at, bt = op_a.upper() == "T", op_b.upper() == "T"
+    if A.dtype != torch.float16 or B.dtype != torch.float16:
+        raise TypeError("A and B must be fp16")
+    M, K = (A.shape[1], A.shape[0]) if at else tuple(A.shape)
+    K2, N = (B.shape[1], B.shape[0]) if bt else tuple(B.shape)
+    if K != K2:
+        raise ValueError(f"inner dimensions differ: op(A) is {M}x{K}, op(B) is {K2}x{N}")
+    o = TLG_OUT_F32 if out == "f32" else TLG_OUT_F16
+    C = _out(C, M, N, torch.float32 if o == TLG_OUT_F32 else torch.float16, A)
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    pc, ldc = _mat(C, "C")
+    cfg = tlg_config(**{k: int(v) for k, v in config.items()}) if config is not None else None
+    epi = TLG_EPI_BIAS_RELU if bias is not None else TLG_EPI_NONE
+    ws_ptr, ws_bytes = (None, 0)
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check(_lib.tlg_gemm_op(M, N, K, TLG_OP_T if at else TLG_OP_N, pa, lda, TLG_OP_T if bt else TLG_OP_N,
+                            pb, ldb, bias.data_ptr() if bias is not None else None, pc, ldc, o, epi,
+                            ctypes.byref(cfg) if cfg is not None else None, ws_ptr, ws_bytes,
+                            _stream_handle(stream, A, B, C)), "tlg_gemm_op")
     return C
 
 

@@ -408,13 +408,15 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor of tcgen05.mma.kind::f16: fp32 D, fp16 A (K-major)
-// and fp16 B (MN-major), shape M x N (x 16).
+// Instruction descriptor of tcgen05.mma.kind::f16: fp32 D, fp16 A and B,
+// shape M x N (x 16), each operand K-major or MN-major in shared memory.
 //   bits 4-5 D format (1 = f32), 7-9 A format (0 = f16), 10-12 B format,
-//   bit 15 A major (0 = K), bit 16 B major (1 = MN), 17-22 N >> 3, 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t make_idesc_f16(int m, int n) {
-  return (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) |
-         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+//   bit 15 A major (0 = K, 1 = MN), bit 16 B major, 17-22 N >> 3, 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t make_idesc_f16(int m, int n, bool a_mn_major = false,
+                                                      bool b_mn_major = true) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
+         (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
 }
 
 }  // namespace tlg

@@ -117,7 +117,7 @@ struct LaunchState {
   int units = 0;
 };
 
-template <int CG, int TN, int STAGES, bool OUT_F16, bool BIAS_RELU>
+template <int CG, int TN, int STAGES, bool OUT_F16, bool BIAS_RELU, bool AT, bool BT>
 struct Variant {
   static constexpr int NH = TN > 256 ? 2 : 1;  // MMA halves per tile
   static constexpr int BN = TN / NH;           // the MMA's N
@@ -153,7 +153,7 @@ struct Variant {
   // or the number of 2-CTA clusters the occupancy calculator admits.
   static tlg_status units(int dev, int sms, int *out) {
     static LaunchState state[kMaxDevices];
-    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH>;
+    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH, AT, BT>;
     std::lock_guard<std::mutex> lock(g_mutex);
     LaunchState &st = state[dev];
     if (!st.ready) {
@@ -188,7 +188,7 @@ struct Variant {
     fill_launch(&cfg, attr, s, overlap_prev);
     cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH>, tmA, tmB, tmC, p);
+        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH, AT, BT>, tmA, tmB, tmC, p);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return TLG_ERR_CUDA;
@@ -203,20 +203,32 @@ struct VariantFns {
                        const GemmParams &, bool, cudaStream_t);
 };
 
-#define TLG_FNS(CG, BN, ST, F16, BR) \
-  VariantFns { Variant<CG, BN, ST, F16, BR>::units, Variant<CG, BN, ST, F16, BR>::launch }
-#define TLG_VARIANT(CG, BN, ST) \
-  { TLG_FNS(CG, BN, ST, false, false), TLG_FNS(CG, BN, ST, true, false), TLG_FNS(CG, BN, ST, true, true) }
+#define TLG_FNS(CG, TN, ST, F16, BR, AT, BT)                   \
+  VariantFns {                                                 \
+    Variant<CG, TN, ST, F16, BR, AT, BT>::units,               \
+        Variant<CG, TN, ST, F16, BR, AT, BT>::launch           \
+  }
+#define TLG_VARIANT(CG, TN, ST, AT, BT)                                             \
+  {                                                                                 \
+    TLG_FNS(CG, TN, ST, false, false, AT, BT), TLG_FNS(CG, TN, ST, true, false, AT, BT), \
+        TLG_FNS(CG, TN, ST, true, true, AT, BT)                                     \
+  }
+#define TLG_LAYOUT(AT, BT)                                                                   \
+  {                                                                                          \
+    TLG_VARIANT(1, 64, 8, AT, BT), TLG_VARIANT(1, 128, 6, AT, BT), TLG_VARIANT(1, 256, 4, AT, BT), \
+        TLG_VARIANT(2, 128, 8, AT, BT), TLG_VARIANT(2, 256, 6, AT, BT),                      \
+        TLG_VARIANT(2, 512, 4, AT, BT)                                                       \
+  }
 
-// [variant, same order as kBuilt][f32 | f16 | f16 bias+ReLU]
-const VariantFns kVariantFns[kNumBuilt][3] = {TLG_VARIANT(1, 64, 8),  TLG_VARIANT(1, 128, 6),
-                                              TLG_VARIANT(1, 256, 4),  TLG_VARIANT(2, 128, 8),
-                                              TLG_VARIANT(2, 256, 6),  TLG_VARIANT(2, 512, 4)};
+// [operand layout: A^T * 2 + B^T][variant, same order as kBuilt][f32 | f16 | f16 bias+ReLU]
+const VariantFns kVariantFns[4][kNumBuilt][3] = {TLG_LAYOUT(false, false), TLG_LAYOUT(false, true),
+                                                 TLG_LAYOUT(true, false), TLG_LAYOUT(true, true)};
+#undef TLG_LAYOUT
 #undef TLG_VARIANT
 #undef TLG_FNS
 
-const VariantFns &fns_for(int idx, bool f16, bool bias_relu) {
-  return kVariantFns[idx][!f16 ? 0 : (bias_relu ? 2 : 1)];
+const VariantFns &fns_for(int idx, bool f16, bool bias_relu, bool at = false, bool bt = false) {
+  return kVariantFns[(at ? 2 : 0) + (bt ? 1 : 0)][idx][!f16 ? 0 : (bias_relu ? 2 : 1)];
 }
 
 // --------------------------------------------------------------------------- schedule
@@ -277,8 +289,10 @@ struct Resolved {
 // Choose (or check) the kernel variant and the schedule.  Shapes are ranked by
 // k-blocks on the critical path times the per-k-block time of the tile (tile
 // area over its sustained fraction of the MMA peak, per SM).
+// at / bt select the operand-layout instantiation whose launch attributes are
+// prepared (the schedule itself does not depend on the layout).
 tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, bool bias_relu,
-                   const tlg_config *req, size_t ws_bytes, Resolved *out) {
+                   bool at, bool bt, const tlg_config *req, size_t ws_bytes, Resolved *out) {
   const int num_kb = static_cast<int>((K + kBK - 1) / kBK);
   tlg_config r = {};
   if (req != nullptr) r = *req;
@@ -296,7 +310,7 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
     if (r.stages != 0 && r.stages != k.stages) continue;
     shape_exists = true;
     int resident = 0;
-    const tlg_status us = fns_for(i, f16, bias_relu).units(dev, sms, &resident);
+    const tlg_status us = fns_for(i, f16, bias_relu, at, bt).units(dev, sms, &resident);
     if (us != TLG_OK) return us;
     if (r.max_ctas > 0) resident = std::max(1, std::min(resident, r.max_ctas / k.cta_group));
     const int64_t tile_m = 128 * k.cta_group;
@@ -360,9 +374,11 @@ tlg_status launch_fill(void *C, int64_t ldc, const void *bias, int M, int N, cud
 }
 
 // Host-only argument checks shared by every entry point; nothing here touches the GPU.
-tlg_status check_args(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
-                      int64_t ldb, const void *bias, const void *C, int64_t ldc, tlg_out out,
-                      tlg_epilogue epi) {
+// at / bt: A stored K x M (lda >= M), B stored N x K (ldb >= K), the product
+// using their transposes.
+tlg_status check_args(int64_t M, int64_t N, int64_t K, bool at, const void *A, int64_t lda,
+                      bool bt, const void *B, int64_t ldb, const void *bias, const void *C,
+                      int64_t ldc, tlg_out out, tlg_epilogue epi) {
   if (out != TLG_OUT_F32 && out != TLG_OUT_F16) return TLG_ERR_INVALID_ARG;
   if (epi != TLG_EPI_NONE && epi != TLG_EPI_BIAS_RELU) return TLG_ERR_INVALID_ARG;
   if (epi == TLG_EPI_BIAS_RELU && out != TLG_OUT_F16) return TLG_ERR_UNSUPPORTED;
@@ -375,7 +391,8 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, const void *A, int64_t ld
   if (M == 0 || N == 0) return TLG_OK;
   const int64_t osz = out == TLG_OUT_F32 ? 4 : 2;
   if (C == nullptr || ldc < N) return TLG_ERR_INVALID_ARG;
-  if (K > 0 && (A == nullptr || B == nullptr || lda < K || ldb < N)) return TLG_ERR_INVALID_ARG;
+  if (K > 0 && (A == nullptr || B == nullptr || lda < (at ? M : K) || ldb < (bt ? K : N)))
+    return TLG_ERR_INVALID_ARG;
   if (!aligned16(C) || (ldc * osz) % 16 != 0) return TLG_ERR_ALIGNMENT;
   if (bias != nullptr && !aligned16(bias)) return TLG_ERR_ALIGNMENT;
   if (K > 0 && (!aligned16(A) || !aligned16(B) || (lda * 2) % 16 != 0 || (ldb * 2) % 16 != 0))
@@ -386,8 +403,14 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, const void *A, int64_t ld
   extent(C, M, N, ldc, osz, &c0, &c1);
   if (K > 0) {
     uintptr_t a0, a1, b0, b1;
-    extent(A, M, K, lda, 2, &a0, &a1);
-    extent(B, K, N, ldb, 2, &b0, &b1);
+    if (at)
+      extent(A, K, M, lda, 2, &a0, &a1);
+    else
+      extent(A, M, K, lda, 2, &a0, &a1);
+    if (bt)
+      extent(B, N, K, ldb, 2, &b0, &b1);
+    else
+      extent(B, K, N, ldb, 2, &b0, &b1);
     if (overlaps(c0, c1, a0, a1) || overlaps(c0, c1, b0, b1)) return TLG_ERR_INVALID_ARG;
   }
   if (bias != nullptr) {
@@ -398,11 +421,11 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, const void *A, int64_t ld
 }
 
 // ws/ws_bytes: scratch for the split-K tail (nullptr/0: none).
-tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
-                     int64_t ldb, const void *bias, void *C, int64_t ldc, tlg_out out,
-                     tlg_epilogue epi, const tlg_config *req, void *ws, size_t ws_bytes,
-                     void *stream) {
-  const tlg_status hs = check_args(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epi);
+tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, int64_t lda,
+                     bool bt, const void *B, int64_t ldb, const void *bias, void *C, int64_t ldc,
+                     tlg_out out, tlg_epilogue epi, const tlg_config *req, void *ws,
+                     size_t ws_bytes, void *stream) {
+  const tlg_status hs = check_args(M, N, K, at, A, lda, bt, B, ldb, bias, C, ldc, out, epi);
   if (hs != TLG_OK || M == 0 || N == 0) return hs;
   const int64_t osz = out == TLG_OUT_F32 ? 4 : 2;
   if (ws == nullptr) ws_bytes = 0;
@@ -414,8 +437,8 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
     if (overlaps(c0, c1, w0, w0 + ws_bytes)) return TLG_ERR_INVALID_ARG;
     if (K > 0) {
       uintptr_t a0, a1, b0, b1;
-      extent(A, M, K, lda, 2, &a0, &a1);
-      extent(B, K, N, ldb, 2, &b0, &b1);
+      extent(A, at ? K : M, at ? M : K, lda, 2, &a0, &a1);
+      extent(B, bt ? N : K, bt ? K : N, ldb, 2, &b0, &b1);
       if (overlaps(w0, w0 + ws_bytes, a0, a1) || overlaps(w0, w0 + ws_bytes, b0, b1))
         return TLG_ERR_INVALID_ARG;
     }
@@ -442,18 +465,24 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
   }
 
   Resolved rv;
-  const tlg_status rs = resolve(dev, info.sm_count, M, N, K, f16, br, req, ws_bytes, &rv);
+  const tlg_status rs = resolve(dev, info.sm_count, M, N, K, f16, br, at, bt, req, ws_bytes, &rv);
   if (rs != TLG_OK) return rs;
   if (rv.sched.workspace > ws_bytes) return TLG_ERR_INVALID_ARG;  // a forced split needs scratch
 
-  // A: K x M boxes of 64 x 128; B: N x K boxes of 64 x 64; C: 32-row boxes of 128 bytes.
+  // Boxes (inner x outer, elements): A 64 k x 128 rows, or 64 m x 64 k when
+  // stored transposed; B 64 n x 64 k, or 64 k x (columns per CTA) when stored
+  // transposed; C 128 bytes x 32 rows.
   CUtensorMap tmA, tmB, tmC;
-  const CUtensorMapDataType c_type =
-      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  if (!encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, A, uint64_t(K), uint64_t(M),
-                 uint64_t(lda) * 2, kBK, kBM) ||
-      !encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, B, uint64_t(N), uint64_t(K),
-                 uint64_t(ldb) * 2, 64, kBK) ||
+  const CUtensorMapDataType h16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType c_type = f16 ? h16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const uint32_t b_rows_per_cta =
+      static_cast<uint32_t>((rv.cfg.block_n > 256 ? 256 : rv.cfg.block_n) / rv.cfg.cta_group);
+  const bool a_ok = at ? encode_2d(&tmA, h16, A, uint64_t(M), uint64_t(K), uint64_t(lda) * 2, 64, kBK)
+                       : encode_2d(&tmA, h16, A, uint64_t(K), uint64_t(M), uint64_t(lda) * 2, kBK, kBM);
+  const bool b_ok = bt ? encode_2d(&tmB, h16, B, uint64_t(K), uint64_t(N), uint64_t(ldb) * 2, kBK,
+                                   b_rows_per_cta)
+                       : encode_2d(&tmB, h16, B, uint64_t(N), uint64_t(K), uint64_t(ldb) * 2, 64, kBK);
+  if (!a_ok || !b_ok ||
       !encode_2d(&tmC, c_type, C, uint64_t(N), uint64_t(M), uint64_t(ldc) * osz,
                  uint32_t(128 / osz), 32))
     return TLG_ERR_CUDA;
@@ -474,7 +503,8 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda
   p.counters = static_cast<uint32_t *>(ws);
   p.ws = ws != nullptr ? reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes)
                        : nullptr;
-  return fns_for(rv.idx, f16, br).launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
+  return fns_for(rv.idx, f16, br, at, bt)
+      .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
 }
 
 // ---------------------------------------------------------------- allocation-free scratch
@@ -527,8 +557,8 @@ tlg_status resolve_public(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_epil
   const tlg_status ds = current_device(&dev, &info);
   if (ds != TLG_OK) return ds;
   return resolve(dev, info.sm_count, std::max<int64_t>(M, 1), std::max<int64_t>(N, 1),
-                 std::max<int64_t>(K, 1), out == TLG_OUT_F16, epilogue == TLG_EPI_BIAS_RELU, req,
-                 ws_bytes, rv);
+                 std::max<int64_t>(K, 1), out == TLG_OUT_F16, epilogue == TLG_EPI_BIAS_RELU, false,
+                 false, req, ws_bytes, rv);
 }
 
 }  // namespace
@@ -537,30 +567,40 @@ extern "C" {
 
 tlg_status tlg_gemm_f16f32(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                            const void *B, int64_t ldb, float *C, int64_t ldc, void *stream) {
-  return gemm_impl(M, N, K, A, lda, B, ldb, nullptr, C, ldc, TLG_OUT_F32, TLG_EPI_NONE, nullptr,
-                   nullptr, 0, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, nullptr, C, ldc, TLG_OUT_F32,
+                   TLG_EPI_NONE, nullptr, nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_f16f16(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                            const void *B, int64_t ldb, void *C, int64_t ldc, void *stream) {
-  return gemm_impl(M, N, K, A, lda, B, ldb, nullptr, C, ldc, TLG_OUT_F16, TLG_EPI_NONE, nullptr,
-                   nullptr, 0, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, nullptr, C, ldc, TLG_OUT_F16,
+                   TLG_EPI_NONE, nullptr, nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_bias_relu_f16(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                                   const void *B, int64_t ldb, const void *bias, void *C,
                                   int64_t ldc, void *stream) {
   if (bias == nullptr && M > 0 && N > 0) return TLG_ERR_INVALID_ARG;
-  return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, TLG_OUT_F16, TLG_EPI_BIAS_RELU, nullptr,
-                   nullptr, 0, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, TLG_OUT_F16,
+                   TLG_EPI_BIAS_RELU, nullptr, nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
                        int64_t ldb, const void *bias, void *C, int64_t ldc, tlg_out out,
                        tlg_epilogue epilogue, const tlg_config *config, void *workspace,
                        size_t workspace_bytes, void *stream) {
-  return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, workspace,
-                   workspace_bytes, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, out, epilogue, config,
+                   workspace, workspace_bytes, stream);
+}
+
+tlg_status tlg_gemm_op(int64_t M, int64_t N, int64_t K, tlg_op op_a, const void *A, int64_t lda,
+                       tlg_op op_b, const void *B, int64_t ldb, const void *bias, void *C,
+                       int64_t ldc, tlg_out out, tlg_epilogue epilogue, const tlg_config *config,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+  if ((op_a != TLG_OP_N && op_a != TLG_OP_T) || (op_b != TLG_OP_N && op_b != TLG_OP_T))
+    return TLG_ERR_INVALID_ARG;
+  return gemm_impl(M, N, K, op_a == TLG_OP_T, A, lda, op_b == TLG_OP_T, B, ldb, bias, C, ldc, out,
+                   epilogue, config, workspace, workspace_bytes, stream);
 }
 
 tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
@@ -569,8 +609,8 @@ tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K, const void *A, i
                                void *stream) {
   const bool split = config != nullptr && config->split_k >= 2;
   if (!split)  // no scratch needed: exactly tlg_gemm_ex without a workspace
-    return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, nullptr, 0,
-                     stream);
+    return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, out, epilogue, config,
+                     nullptr, 0, stream);
   // Reject a schedule whose scratch would not fit before touching anything.
   if (M > 0 && N > 0 && K > 0) {
     Resolved rv;
@@ -587,8 +627,8 @@ tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K, const void *A, i
     cudaGetLastError();
     return TLG_ERR_CUDA;
   }
-  return gemm_impl(M, N, K, A, lda, B, ldb, bias, C, ldc, out, epilogue, config, scratch,
-                   kStaticScratchBytes, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, out, epilogue, config,
+                   scratch, kStaticScratchBytes, stream);
 }
 
 tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,

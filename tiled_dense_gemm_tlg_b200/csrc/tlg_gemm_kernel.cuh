@@ -209,7 +209,14 @@ __device__ __forceinline__ void store_row_tail(const GemmParams &p, int row, int
 // main loop.  NH == 2: each tile is 2*BN wide and fills TMEM with two
 // BN-column halves; the epilogue hands half 0 back before draining half 1, so
 // the next tile's MMAs into half 0 start while half 1 is still being stored.
-template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU, int NH = 1>
+//
+// AT / BT select how the operands are stored.  AT == false: A is M x K
+// row-major (K contiguous, a K-major operand); AT == true: the stored matrix
+// is K x M row-major and the product uses its transpose (an MN-major
+// operand).  BT == false: B is K x N row-major (MN-major operand); BT == true:
+// the stored matrix is N x K row-major, transposed (K-major operand).
+template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU, int NH = 1, bool AT = false,
+          bool BT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB,
@@ -300,26 +307,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t a_dst = smem_u32(sA + stage * Plan::kABytes);
         const uint32_t b_dst = smem_u32(sB + stage * Plan::kBBytes);
+        uint32_t bar;
         if constexpr (CG == 1) {
-          mbar_arrive_expect_tx(full_bar(stage), Plan::kStageBytes);
-          tma_load_2d(a_dst, &tmA, full_bar(stage), kb * kBK, a_row);
-#pragma unroll
-          for (int h = 0; h < NH; ++h)
-#pragma unroll
-            for (int c = 0; c < Plan::kBNc / 64; ++c)
-              tma_load_2d(b_dst + h * Plan::kHalfBBytes + c * 8192, &tmB, full_bar(stage),
-                          b_col + h * BN + c * 64, kb * kBK);
+          bar = full_bar(stage);
+          mbar_arrive_expect_tx(bar, Plan::kStageBytes);
         } else {
           // The leader's full barrier counts the bytes of both CTAs' loads.
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * Plan::kStageBytes);
-          const uint32_t bar = mapa_shared(full_bar(stage), 0);
-          tma_load_2d_pair(a_dst, &tmA, bar, kb * kBK, a_row);
+          bar = mapa_shared(full_bar(stage), 0);
+        }
+        auto load = [&](uint32_t dst, const CUtensorMap *tm, int32_t x, int32_t y) {
+          if constexpr (CG == 1)
+            tma_load_2d(dst, tm, bar, x, y);
+          else
+            tma_load_2d_pair(dst, tm, bar, x, y);
+        };
+        // A tile: 128 rows x 64 k.  K-major: one box; MN-major: two 64-row boxes.
+        if constexpr (!AT) {
+          load(a_dst, &tmA, kb * kBK, a_row);
+        } else {
+          load(a_dst, &tmA, a_row, kb * kBK);
+          load(a_dst + 8192, &tmA, a_row + 64, kb * kBK);
+        }
+        // B slice of each half: kBNc columns x 64 k.  MN-major: 64-column boxes;
+        // K-major: one box of kBNc rows.
 #pragma unroll
-          for (int h = 0; h < NH; ++h)
+        for (int h = 0; h < NH; ++h) {
+          if constexpr (!BT) {
 #pragma unroll
             for (int c = 0; c < Plan::kBNc / 64; ++c)
-              tma_load_2d_pair(b_dst + h * Plan::kHalfBBytes + c * 8192, &tmB, bar,
-                               b_col + h * BN + c * 64, kb * kBK);
+              load(b_dst + h * Plan::kHalfBBytes + c * 8192, &tmB, b_col + h * BN + c * 64,
+                   kb * kBK);
+          } else {
+            load(b_dst + h * Plan::kHalfBBytes, &tmB, kb * kBK, b_col + h * BN);
+          }
         }
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -353,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------------------- MMA issuer (leader CTA)
-    constexpr uint32_t idesc = make_idesc_f16(kTileM, BN);
+    constexpr uint32_t idesc = make_idesc_f16(kTileM, BN, AT, !BT);
     int stage = 0;
     uint32_t phase = 0;
     // Accumulator slots are the two BN-column halves of TMEM.  NH == 1: tiles
@@ -393,9 +414,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((NH == 1 ? acc : h) * BN);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
-            const uint64_t bdesc =
-                smem_desc_sw128(b0 + h * Plan::kHalfBBytes + kk * 16 * 128, 8192, 1024);
+            // K-major: 16 k = 32 bytes along the swizzled row; MN-major: 16 k
+            // = 16 rows of 128 bytes, 64-element blocks 8192 bytes apart.
+            const uint64_t adesc = !AT ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
+                                       : smem_desc_sw128(a0 + kk * 16 * 128, 8192, 1024);
+            const uint32_t bh = b0 + h * Plan::kHalfBBytes;
+            const uint64_t bdesc = !BT ? smem_desc_sw128(bh + kk * 16 * 128, 8192, 1024)
+                                       : smem_desc_sw128(bh + kk * 32, 16, 1024);
             mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (kb > w.kb0 || kk > 0) ? 1u : 0u);
           }
         }
