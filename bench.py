@@ -287,6 +287,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layout", default="NN", choices=["NN", "NT", "TN", "TT"],
                     help="op(A), op(B): T = that operand is stored transposed (tlg_gemm_op)")
+    ap.add_argument("--ld-pad", type=int, default=0,
+                    help="extra elements in every row stride (odd: strides TMA cannot describe, "
+                         "served by the plain-load path)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
@@ -307,9 +310,19 @@ def main(argv=None):
         A = A.t().contiguous()  # stored K x M; the product uses its transpose
     if bt:
         B = B.t().contiguous()  # stored N x K
-    dA, dB = A.to(dev), B.to(dev)
+    def padded(x: torch.Tensor, pad: int) -> torch.Tensor:
+        """x on the device as a view with row stride cols + pad."""
+        if pad == 0:
+            return x.to(dev)
+        buf = torch.empty((x.shape[0], x.shape[1] + pad), dtype=x.dtype, device=dev)
+        view = buf[:, :x.shape[1]]
+        view.copy_(x)
+        return view
+
+    dA, dB = padded(A, args.ld_pad), padded(B, args.ld_pad)
     dbias = bias.to(dev) if bias is not None else None
-    dC = torch.empty((w.M, w.N), dtype=torch.float32 if w.out == "f32" else torch.float16, device=dev)
+    dC = padded(torch.empty((w.M, w.N), dtype=torch.float32 if w.out == "f32" else torch.float16),
+                args.ld_pad)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     override = json.loads(args.config) if args.config else None
     kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu, request=override)
@@ -318,7 +331,7 @@ def main(argv=None):
     ws = tlg.tlg_workspace(ws_bytes, device=dev) if ws_bytes > 0 else None
     plain_name = ("tlg_gemm_bias_relu_f16" if w.bias_relu else
                   ("tlg_gemm_f16f16" if w.out == "f16" else "tlg_gemm_f16f32"))
-    use_op = at or bt
+    use_op = at or bt or args.ld_pad != 0
     use_ex = (ws is not None or override is not None) and not use_op
     entry = "tlg_gemm_op" if use_op else ("tlg_gemm_ex" if use_ex else plain_name)
 
@@ -455,7 +468,9 @@ def main(argv=None):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": dict(workload_config(w, kcfg), entry_point=entry, workspace_bytes=ws_bytes,
-                       layout=args.layout),
+                       layout=args.layout, ld_pad=args.ld_pad,
+                       operand_path=("plain loads/stores (row strides not 16-byte multiples)"
+                                     if (args.ld_pad * 2) % 16 else "TMA")),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "plain_entry_point": plain,
         "gpu_launches": args.steps,
         "clocks": clk,

@@ -28,9 +28,12 @@
  *    NULL means the legacy default stream) and returns.  Calls are
  *    stream-ordered and may be issued from several host threads.
  *  - The library allocates no device memory.
- *  - Alignment (a rule of the TMA engine that loads the tiles): A, B, C and
- *    the bias must be 16-byte aligned, and lda*2, ldb*2 and ldc*sizeof(out)
- *    must be multiples of 16 bytes.  Otherwise TLG_ERR_ALIGNMENT.
+ *  - Alignment: every pointer must be aligned to its element (2 bytes for fp16
+ *    data, 4 for an fp32 C), else TLG_ERR_ALIGNMENT.  The fast path loads and
+ *    stores tiles with the TMA engine, which needs 16-byte aligned bases and
+ *    row strides (lda*2, ldb*2, ldc*sizeof(out)) that are multiples of 16
+ *    bytes; operands that break that rule are loaded by plain loads (several
+ *    times slower) and such a C is written by plain stores.
  *  - Sizes: 0 <= M, N, K <= 2^31 - 257, and ceil(M/128)*ceil(N/64) below 2^31
  *    (larger sizes give TLG_ERR_UNSUPPORTED); lda >= K, ldb >= N, ldc >= N.
  *    M == 0 or N == 0: nothing is written, TLG_OK.  K == 0: the empty sum is

@@ -71,8 +71,8 @@ def test_host_side_rejections_need_no_gpu(lib_path):
     assert f(-1, 8, 8, A, 8, A, 8, A, 8, None) == tlg.TLG_ERR_INVALID_ARG
     assert f(8, 8, 8, None, 8, A, 8, A * 2, 8, None) == tlg.TLG_ERR_INVALID_ARG
     assert f(8, 8, 8, A, 7, A, 8, A * 2, 8, None) == tlg.TLG_ERR_INVALID_ARG
-    assert f(8, 8, 8, A + 2, 8, A, 8, A * 2, 8, None) == tlg.TLG_ERR_ALIGNMENT
-    assert f(8, 8, 12, A, 12, A, 8, A * 2, 8, None) == tlg.TLG_ERR_ALIGNMENT
+    assert f(8, 8, 8, A + 1, 8, A, 8, A * 2, 8, None) == tlg.TLG_ERR_ALIGNMENT  # odd address for fp16
+    assert f(8, 8, 8, A, 8, A, 8, A * 2 + 2, 8, None) == tlg.TLG_ERR_ALIGNMENT  # fp32 C needs 4 bytes
     assert f(8, 8, 8, A, 8, A, 8, A + 64, 8, None) == tlg.TLG_ERR_INVALID_ARG  # C overlaps A
     assert f(0, 8, 8, None, 8, None, 8, None, 8, None) == tlg.TLG_OK  # empty: nothing to do
     assert lib.tlg_gemm_bias_relu_f16(8, 8, 8, A, 8, A, 8, None, A * 2, 8, None) == tlg.TLG_ERR_INVALID_ARG

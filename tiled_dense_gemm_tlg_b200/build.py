@@ -25,7 +25,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtlg.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-O2", "--expt-relaxed-constexpr",
          "-Xptxas", "-v"]
 
 
@@ -52,20 +52,45 @@ def needs_build() -> bool:
     return any(os.path.getmtime(f) > t for f in inputs())
 
 
+def _compile(src: str, obj: str):
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-Xcompiler", "-fPIC", "-c", "-o", obj, src]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    return cmd, res
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every .cu (one translation unit per operand layout, in parallel) and link libtlg.so."""
     if not (force or needs_build()):
         return LIB
+    import concurrent.futures
+
+    import shutil
+    import tempfile
+
+    obj_dir = tempfile.mkdtemp(prefix="tlg_build_")  # objects are intermediates: not kept in the tree
+    srcs = sources()
+    objs = [os.path.join(obj_dir, os.path.basename(s)[:-3] + ".o") for s in srcs]
+    log_lines = []
+    failed = False
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        for (cmd, res) in ex.map(_compile, srcs, objs):
+            log_lines.append(" ".join(cmd) + "\n" + res.stdout + res.stderr)
+            failed = failed or res.returncode != 0
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp, *sources()]
-    res = subprocess.run(cmd, capture_output=True, text=True)
+    if not failed:
+        cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        log_lines.append(" ".join(cmd) + "\n" + res.stdout + res.stderr)
+        failed = res.returncode != 0
+    shutil.rmtree(obj_dir, ignore_errors=True)
     log = os.path.join(PKG, "_build_log.txt")
     with open(log, "w") as f:
-        f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
-    if res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError(f"nvcc failed (exit {res.returncode}); see {log}")
+        f.write("\n".join(log_lines))
+    if failed:
+        sys.stderr.write("\n".join(l for l in log_lines if "error" in l)[-20000:])
+        raise RuntimeError(f"nvcc failed; see {log}")
     if verbose:
-        sys.stderr.write(res.stderr)
+        sys.stderr.write("\n".join(log_lines))
     os.replace(tmp, LIB)
     return LIB
 

@@ -84,7 +84,7 @@ constexpr uint32_t kWaitSuspendNs = 10000000u;
 // time pass.  On the time limit it records the role in the device error word
 // and raises the abort flag so every other role stops waiting too.
 // Returns true only when the phase completed.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
                                             volatile uint32_t *abort_flag, uint64_t limit_ns,
                                             uint32_t role, uint32_t *err_word) {
   const uint64_t t0 = global_timer_ns();

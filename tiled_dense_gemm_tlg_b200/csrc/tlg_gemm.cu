@@ -10,13 +10,12 @@
 #include <mutex>
 
 #include "tlg.h"
-#include "tlg_gemm_kernel.cuh"
+#include "tlg_variants.cuh"
 
 namespace {
 
 using namespace tlg;
 
-constexpr int kMaxDevices = 64;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
 constexpr size_t kCounterBytes = 4096;            // slice counters at the start of a workspace
 constexpr size_t kWorkspaceAlign = 256;
@@ -96,6 +95,7 @@ struct KernelCfg {
   int stages;
   double eff;         // sustained fraction of the MMA peak, relative (ranks tile shapes)
   double exposed_kb;  // k-blocks per tile the main loop waits for the epilogue
+  bool plain_loads;   // also built with the plain-load path (operands TMA cannot describe)
 };
 
 // Kernel variants the library is built with.  A tile is 128*cta_group rows by
@@ -107,128 +107,18 @@ struct KernelCfg {
 // The 512-wide tile moves 25 % fewer operand bytes per FLOP, which under the
 // 1000 W cap buys a higher clock (sustained at 8192^3: 1297 vs 1170 MHz), but
 // its single accumulator leaves part of each epilogue exposed (exposed_kb).
-constexpr KernelCfg kBuilt[] = {{1, 64, 8, 0.35, 0},  {1, 128, 6, 0.60, 0}, {1, 256, 4, 0.90, 0},
-                                {2, 128, 8, 0.60, 0}, {2, 256, 6, 1.00, 0}, {2, 512, 4, 1.07, 8}};
+constexpr KernelCfg kBuilt[] = {{1, 64, 8, 0.35, 0, true},   {1, 128, 6, 0.60, 0, false},
+                                {1, 256, 4, 0.90, 0, false},  {2, 128, 8, 0.60, 0, false},
+                                {2, 256, 6, 1.00, 0, true},   {2, 512, 4, 1.07, 8, false}};
 constexpr int kNumBuilt = sizeof(kBuilt) / sizeof(kBuilt[0]);
+static_assert(kNumBuilt == kNumVariants, "one launcher table entry per built variant");
 
-// Per device and instantiation: kernel attributes set, co-resident work units.
-struct LaunchState {
-  bool ready = false;
-  int units = 0;
-};
-
-template <int CG, int TN, int STAGES, bool OUT_F16, bool BIAS_RELU, bool AT, bool BT>
-struct Variant {
-  static constexpr int NH = TN > 256 ? 2 : 1;  // MMA halves per tile
-  static constexpr int BN = TN / NH;           // the MMA's N
-  using Plan = SmemPlan<CG, BN, STAGES, NH>;
-
-  // attr must hold 2 entries.  With overlap_prev the kernel may start while
-  // the previous kernel in the stream finishes (programmatic stream
-  // serialization); it waits for that kernel before touching global memory.
-  static void fill_launch(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, cudaStream_t s,
-                          bool overlap_prev = false) {
-    *cfg = {};
-    cfg->blockDim = dim3(kThreads, 1, 1);
-    cfg->dynamicSmemBytes = Plan::kDynamicBytes;
-    cfg->stream = s;
-    int n = 0;
-    if (overlap_prev) {
-      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[n].val.programmaticStreamSerializationAllowed = 1;
-      ++n;
-    }
-    if (CG == 2) {
-      attr[n].id = cudaLaunchAttributeClusterDimension;
-      attr[n].val.clusterDim.x = 2;
-      attr[n].val.clusterDim.y = 1;
-      attr[n].val.clusterDim.z = 1;
-      ++n;
-    }
-    cfg->attrs = attr;
-    cfg->numAttrs = n;
-  }
-
-  // Work units (CTAs, or CTA pairs) that can be resident at once: one per SM,
-  // or the number of 2-CTA clusters the occupancy calculator admits.
-  static tlg_status units(int dev, int sms, int *out) {
-    static LaunchState state[kMaxDevices];
-    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH, AT, BT>;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    LaunchState &st = state[dev];
-    if (!st.ready) {
-      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Plan::kDynamicBytes) != cudaSuccess) {
-        cudaGetLastError();
-        return TLG_ERR_CUDA;
-      }
-      int n = sms;
-      if (CG == 2) {
-        cudaLaunchConfig_t cfg;
-        cudaLaunchAttribute attr[2];
-        fill_launch(&cfg, attr, nullptr);
-        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-        if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
-          cudaGetLastError();
-          return TLG_ERR_CUDA;
-        }
-      }
-      st.units = n;
-      st.ready = true;
-    }
-    *out = st.units;
-    return TLG_OK;
-  }
-
-  static tlg_status launch(int units, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                           const CUtensorMap &tmC, const GemmParams &p, bool overlap_prev,
-                           cudaStream_t s) {
-    cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute attr[2];
-    fill_launch(&cfg, attr, s, overlap_prev);
-    cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
-    const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH, AT, BT>, tmA, tmB, tmC, p);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return TLG_ERR_CUDA;
-    }
-    return TLG_OK;
-  }
-};
-
-struct VariantFns {
-  tlg_status (*units)(int, int, int *);
-  tlg_status (*launch)(int, const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                       const GemmParams &, bool, cudaStream_t);
-};
-
-#define TLG_FNS(CG, TN, ST, F16, BR, AT, BT)                   \
-  VariantFns {                                                 \
-    Variant<CG, TN, ST, F16, BR, AT, BT>::units,               \
-        Variant<CG, TN, ST, F16, BR, AT, BT>::launch           \
-  }
-#define TLG_VARIANT(CG, TN, ST, AT, BT)                                             \
-  {                                                                                 \
-    TLG_FNS(CG, TN, ST, false, false, AT, BT), TLG_FNS(CG, TN, ST, true, false, AT, BT), \
-        TLG_FNS(CG, TN, ST, true, true, AT, BT)                                     \
-  }
-#define TLG_LAYOUT(AT, BT)                                                                   \
-  {                                                                                          \
-    TLG_VARIANT(1, 64, 8, AT, BT), TLG_VARIANT(1, 128, 6, AT, BT), TLG_VARIANT(1, 256, 4, AT, BT), \
-        TLG_VARIANT(2, 128, 8, AT, BT), TLG_VARIANT(2, 256, 6, AT, BT),                      \
-        TLG_VARIANT(2, 512, 4, AT, BT)                                                       \
-  }
-
-// [operand layout: A^T * 2 + B^T][variant, same order as kBuilt][f32 | f16 | f16 bias+ReLU]
-const VariantFns kVariantFns[4][kNumBuilt][3] = {TLG_LAYOUT(false, false), TLG_LAYOUT(false, true),
-                                                 TLG_LAYOUT(true, false), TLG_LAYOUT(true, true)};
-#undef TLG_LAYOUT
-#undef TLG_VARIANT
-#undef TLG_FNS
-
-const VariantFns &fns_for(int idx, bool f16, bool bias_relu, bool at = false, bool bt = false) {
-  return kVariantFns[(at ? 2 : 0) + (bt ? 1 : 0)][idx][!f16 ? 0 : (bias_relu ? 2 : 1)];
+const VariantFns &fns_for(int idx, bool f16, bool bias_relu, bool at = false, bool bt = false,
+                          bool plain = false) {
+  static const LayoutTables *const layouts[4] = {&kLayoutNN, &kLayoutNT, &kLayoutTN, &kLayoutTT};
+  const LayoutTables &t = *layouts[(at ? 2 : 0) + (bt ? 1 : 0)];
+  const int kind = !f16 ? 0 : (bias_relu ? 2 : 1);
+  return plain ? t.plain[idx][kind] : t.tma[idx][kind];
 }
 
 // --------------------------------------------------------------------------- schedule
@@ -292,7 +182,8 @@ struct Resolved {
 // at / bt select the operand-layout instantiation whose launch attributes are
 // prepared (the schedule itself does not depend on the layout).
 tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, bool bias_relu,
-                   bool at, bool bt, const tlg_config *req, size_t ws_bytes, Resolved *out) {
+                   bool at, bool bt, bool plain, const tlg_config *req, size_t ws_bytes,
+                   Resolved *out) {
   const int num_kb = static_cast<int>((K + kBK - 1) / kBK);
   tlg_config r = {};
   if (req != nullptr) r = *req;
@@ -308,9 +199,10 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
     if (r.cta_group != 0 && r.cta_group != k.cta_group) continue;
     if (r.block_n != 0 && r.block_n != k.block_n) continue;
     if (r.stages != 0 && r.stages != k.stages) continue;
+    if (plain && !k.plain_loads) continue;
     shape_exists = true;
     int resident = 0;
-    const tlg_status us = fns_for(i, f16, bias_relu, at, bt).units(dev, sms, &resident);
+    const tlg_status us = fns_for(i, f16, bias_relu, at, bt, plain).units(dev, sms, &resident);
     if (us != TLG_OK) return us;
     if (r.max_ctas > 0) resident = std::max(1, std::min(resident, r.max_ctas / k.cta_group));
     const int64_t tile_m = 128 * k.cta_group;
@@ -393,10 +285,12 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, bool at, const void *A, i
   if (C == nullptr || ldc < N) return TLG_ERR_INVALID_ARG;
   if (K > 0 && (A == nullptr || B == nullptr || lda < (at ? M : K) || ldb < (bt ? K : N)))
     return TLG_ERR_INVALID_ARG;
-  if (!aligned16(C) || (ldc * osz) % 16 != 0) return TLG_ERR_ALIGNMENT;
-  if (bias != nullptr && !aligned16(bias)) return TLG_ERR_ALIGNMENT;
-  if (K > 0 && (!aligned16(A) || !aligned16(B) || (lda * 2) % 16 != 0 || (ldb * 2) % 16 != 0))
-    return TLG_ERR_ALIGNMENT;
+  // Only element alignment is required; strides and bases TMA cannot describe
+  // take the plain-load / plain-store paths.
+  auto misaligned = [](const void *q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) % a) != 0; };
+  if (misaligned(C, static_cast<uintptr_t>(osz))) return TLG_ERR_ALIGNMENT;
+  if (bias != nullptr && misaligned(bias, 2)) return TLG_ERR_ALIGNMENT;
+  if (K > 0 && (misaligned(A, 2) || misaligned(B, 2))) return TLG_ERR_ALIGNMENT;
   if (ldc > (int64_t(1) << 36) || lda > (int64_t(1) << 36) || ldb > (int64_t(1) << 36))
     return TLG_ERR_UNSUPPORTED;
   uintptr_t c0, c1;
@@ -464,27 +358,34 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
     return launch_fill<true, false>(C, ldc, bias, int(M), int(N), s);
   }
 
+  // TMA needs 16-byte aligned bases and row strides.
+  const bool plain = !(aligned16(A) && aligned16(B) && (lda * 2) % 16 == 0 && (ldb * 2) % 16 == 0);
+  const bool c_plain = !(aligned16(C) && (ldc * osz) % 16 == 0);
   Resolved rv;
-  const tlg_status rs = resolve(dev, info.sm_count, M, N, K, f16, br, at, bt, req, ws_bytes, &rv);
+  const tlg_status rs =
+      resolve(dev, info.sm_count, M, N, K, f16, br, at, bt, plain, req, ws_bytes, &rv);
   if (rs != TLG_OK) return rs;
   if (rv.sched.workspace > ws_bytes) return TLG_ERR_INVALID_ARG;  // a forced split needs scratch
 
   // Boxes (inner x outer, elements): A 64 k x 128 rows, or 64 m x 64 k when
   // stored transposed; B 64 n x 64 k, or 64 k x (columns per CTA) when stored
   // transposed; C 128 bytes x 32 rows.
-  CUtensorMap tmA, tmB, tmC;
+  // (Maps a path does not use stay zeroed and are never read by the kernel.)
+  CUtensorMap tmA = {}, tmB = {}, tmC = {};
   const CUtensorMapDataType h16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const CUtensorMapDataType c_type = f16 ? h16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const uint32_t b_rows_per_cta =
       static_cast<uint32_t>((rv.cfg.block_n > 256 ? 256 : rv.cfg.block_n) / rv.cfg.cta_group);
-  const bool a_ok = at ? encode_2d(&tmA, h16, A, uint64_t(M), uint64_t(K), uint64_t(lda) * 2, 64, kBK)
-                       : encode_2d(&tmA, h16, A, uint64_t(K), uint64_t(M), uint64_t(lda) * 2, kBK, kBM);
-  const bool b_ok = bt ? encode_2d(&tmB, h16, B, uint64_t(K), uint64_t(N), uint64_t(ldb) * 2, kBK,
-                                   b_rows_per_cta)
-                       : encode_2d(&tmB, h16, B, uint64_t(N), uint64_t(K), uint64_t(ldb) * 2, 64, kBK);
-  if (!a_ok || !b_ok ||
-      !encode_2d(&tmC, c_type, C, uint64_t(N), uint64_t(M), uint64_t(ldc) * osz,
-                 uint32_t(128 / osz), 32))
+  if (!plain) {
+    const bool a_ok = at ? encode_2d(&tmA, h16, A, uint64_t(M), uint64_t(K), uint64_t(lda) * 2, 64, kBK)
+                         : encode_2d(&tmA, h16, A, uint64_t(K), uint64_t(M), uint64_t(lda) * 2, kBK, kBM);
+    const bool b_ok = bt ? encode_2d(&tmB, h16, B, uint64_t(K), uint64_t(N), uint64_t(ldb) * 2, kBK,
+                                     b_rows_per_cta)
+                         : encode_2d(&tmB, h16, B, uint64_t(N), uint64_t(K), uint64_t(ldb) * 2, 64, kBK);
+    if (!a_ok || !b_ok) return TLG_ERR_CUDA;
+  }
+  if (!c_plain && !encode_2d(&tmC, c_type, C, uint64_t(N), uint64_t(M), uint64_t(ldc) * osz,
+                             uint32_t(128 / osz), 32))
     return TLG_ERR_CUDA;
 
   GemmParams p;
@@ -503,7 +404,13 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   p.counters = static_cast<uint32_t *>(ws);
   p.ws = ws != nullptr ? reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes)
                        : nullptr;
-  return fns_for(rv.idx, f16, br, at, bt)
+  p.A = static_cast<const __half *>(A);
+  p.B = static_cast<const __half *>(B);
+  p.lda = lda;
+  p.ldb = ldb;
+  p.c_plain = c_plain ? 1 : 0;
+  p.bias_aligned = (bias != nullptr && aligned16(bias)) ? 1 : 0;
+  return fns_for(rv.idx, f16, br, at, bt, plain)
       .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
 }
 
@@ -558,10 +465,30 @@ tlg_status resolve_public(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_epil
   if (ds != TLG_OK) return ds;
   return resolve(dev, info.sm_count, std::max<int64_t>(M, 1), std::max<int64_t>(N, 1),
                  std::max<int64_t>(K, 1), out == TLG_OUT_F16, epilogue == TLG_EPI_BIAS_RELU, false,
-                 false, req, ws_bytes, rv);
+                 false, false, req, ws_bytes, rv);
 }
 
 }  // namespace
+
+namespace tlg {
+
+// One thread waits on a barrier that nothing signals; the bounded wait gives
+// up after limit_ns, records the timeout and the kernel returns normally.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_word;
+  if (threadIdx.x == 0) {
+    abort_word = 0u;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    mbar_wait(smem_u32(&bar), 0, &abort_word, limit_ns, kRoleSelftest, &g_device_error);
+  }
+}
+
+
+TLG_DEFINE_ERROR_WORD_READER(error_word_host)
+
+}  // namespace tlg
 
 extern "C" {
 
@@ -660,17 +587,16 @@ tlg_status tlg_device_error(int clear, uint32_t *code_out) {
     cudaGetLastError();
     return TLG_ERR_CUDA;
   }
+  // Every translation unit's kernels report into that unit's own word.
+  tlg_status (*const readers[])(bool, uint32_t *) = {tlg::error_word_host, tlg::error_word_nn,
+                                                     tlg::error_word_nt, tlg::error_word_tn,
+                                                     tlg::error_word_tt};
   uint32_t v = 0;
-  if (cudaMemcpyFromSymbol(&v, tlg::g_device_error, sizeof(v)) != cudaSuccess) {
-    cudaGetLastError();
-    return TLG_ERR_CUDA;
-  }
-  if (clear && v != 0) {
-    const uint32_t zero = 0;
-    if (cudaMemcpyToSymbol(tlg::g_device_error, &zero, sizeof(zero)) != cudaSuccess) {
-      cudaGetLastError();
-      return TLG_ERR_CUDA;
-    }
+  for (auto read : readers) {
+    uint32_t w = 0;
+    const tlg_status rs = read(clear != 0, &w);
+    if (rs != TLG_OK) return rs;
+    v |= w;
   }
   if (code_out) *code_out = v;
   return v ? TLG_ERR_TIMEOUT : TLG_OK;

@@ -36,9 +36,16 @@ constexpr int kBM = 128;  // tile rows per CTA (TMEM lanes)
 constexpr int kBK = 64;   // k-block: 64 fp16 = one 128-byte swizzle row
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kEpiWarps);  // producer warp, MMA warp, epilogue warps
+// Operands TMA cannot describe (a row stride or base not 16-byte aligned) are
+// loaded by kLoaderWarps extra warps with plain loads instead.
+constexpr int kLoaderWarps = 4;
+constexpr int kThreadsLsu = kThreads + 32 * kLoaderWarps;
 constexpr uint32_t kStageOutBytes = 32 * 128;   // one TMA store box: 32 rows x 128 bytes
 
-__device__ uint32_t g_device_error;
+// Device error word (see tlg_device_error in tlg.h); internal linkage, so
+// every translation unit that includes this header has its own copy, and the
+// host side reads them all.
+static __device__ uint32_t g_device_error;
 
 // Shared-memory plan of one CTA.  CG CTAs (1 or 2) compute one tile of
 // 128*CG rows by NH*BN columns (BN = the MMA's N; NH = 1, or 2 for a tile of
@@ -80,6 +87,12 @@ struct GemmParams {
   int tail_items;
   float *ws;           // fp32 partial sums of the tail slices
   uint32_t *counters;  // per (tail tile, CTA of the group, epilogue warp): slices written so far
+  // Plain-load path (kernels built with LSU): the stored operands.
+  const __half *A;
+  const __half *B;
+  int64_t lda, ldb;
+  int c_plain;       // C cannot be written by TMA (base or row stride not 16-byte aligned)
+  int bias_aligned;  // the bias may be read 16 bytes at a time
 };
 
 // One unit of work: a tile, or one k-slice of a tail tile.
@@ -138,8 +151,8 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int gro
 // Adds bias[col0 + j] (j < 32) to v and applies the ReLU.  Bias entries at
 // columns >= N are not read (those outputs are clipped by the store).
 __device__ __forceinline__ void bias_relu_32(const __half *__restrict__ bias, int col0, int N,
-                                             float (&v)[32]) {
-  if (col0 + 32 <= N) {
+                                             bool aligned, float (&v)[32]) {
+  if (aligned && col0 + 32 <= N) {
     const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -204,6 +217,55 @@ __device__ __forceinline__ void store_row_tail(const GemmParams &p, int row, int
   }
 }
 
+// ------------------------------------------------------------------ plain-load path
+
+// Elements (row, col) and (row, col + 1) of a row-major fp16 matrix with
+// `rows` x `cols` valid elements and row stride ld, packed low/high; elements
+// outside the matrix read as 0 (as the TMA path's out-of-range fill).  Any
+// 2-byte alignment is fine.
+// Predicated read-only global load of one 16-bit element (0 when !pred).
+// Volatile, like the shared-memory stores, so a batch's loads stay in program
+// order ahead of its stores and are all in flight together.
+__device__ __forceinline__ uint32_t ld_u16_pred(const void *ptr, bool pred) {
+  uint16_t x;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %2, 0;\n\t"
+      "mov.u16 %0, 0;\n\t"
+      "@p ld.global.nc.u16 %0, [%1];\n\t}"
+      : "=h"(x)
+      : "l"(ptr), "r"(static_cast<uint32_t>(pred)));
+  return x;
+}
+
+__device__ __forceinline__ uint32_t load_pair(const __half *base, int row, int col, int64_t ld,
+                                              int rows, int cols) {
+  const unsigned short *q = reinterpret_cast<const unsigned short *>(base) +
+                            static_cast<int64_t>(row < rows ? row : 0) * ld + col;
+  const uint32_t lo = ld_u16_pred(q, row < rows && col < cols);
+  const uint32_t hi = ld_u16_pred(q + 1, row < rows && col + 1 < cols);
+  return lo | (hi << 16);
+}
+
+// No memory clobber: the loads of a batch may be issued ahead of its stores;
+// the async-proxy fence that follows a stage (volatile, with a clobber) keeps
+// every store before the barrier arrive.
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+
+// Byte offsets in the 128-byte-swizzled operand layouts the tensor core reads
+// (the same layouts the TMA path writes).  K-major: one 128-byte row of 64 k
+// per M/N index.  MN-major: 64-element blocks of 64 rows (one per k), 8 KB apart.
+__device__ __forceinline__ uint32_t kmajor_offset(int mn, int k) {
+  return static_cast<uint32_t>(mn * 128 + ((((k >> 3) ^ (mn & 7))) << 4) + (k & 7) * 2);
+}
+
+__device__ __forceinline__ uint32_t mnmajor_offset(int mn, int k) {
+  return static_cast<uint32_t>((mn >> 6) * 8192 + k * 128 + (((((mn & 63) >> 3) ^ (k & 7))) << 4) +
+                               (mn & 7) * 2);
+}
+
 // NH == 1: each tile is one BN-wide accumulator and two accumulators
 // alternate in TMEM, so the epilogue of one tile overlaps the next tile's
 // main loop.  NH == 2: each tile is 2*BN wide and fills TMEM with two
@@ -215,9 +277,13 @@ __device__ __forceinline__ void store_row_tail(const GemmParams &p, int row, int
 // is K x M row-major and the product uses its transpose (an MN-major
 // operand).  BT == false: B is K x N row-major (MN-major operand); BT == true:
 // the stored matrix is N x K row-major, transposed (K-major operand).
+//
+// LSU: the operands are loaded by kLoaderWarps extra warps with 2-byte global
+// loads into the same swizzled shared-memory layouts, for strides and bases
+// the TMA unit cannot describe; the tensor-core pipeline is unchanged.
 template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU, int NH = 1, bool AT = false,
-          bool BT = false>
-__global__ void __launch_bounds__(kThreads, 1)
+          bool BT = false, bool LSU = false>
+__global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
@@ -226,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kTileN = BN * NH;
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
   static_assert(NH == 1 || NH == 2, "one accumulator per tile, or two halves");
+  static_assert(!LSU || NH == 1, "the plain-load path is built for one-accumulator tiles");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
 
   extern __shared__ uint8_t smem_raw[];
@@ -257,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), LSU ? kLoaderWarps * CG : 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -267,9 +334,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_mbar_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    tma_prefetch_desc(&tmC);
+    if constexpr (!LSU) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+    }
+    if (!p.c_plain) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc<CG>(smem_u32(tmem_holder), Plan::kTmemCols);
@@ -289,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   grid_dependency_wait();
   grid_launch_dependents();
 
-  if (warp == 0 && lane == 0) {
+  if (!LSU && warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- producer (every CTA)
     int stage = 0;
     uint32_t phase = 0;
@@ -445,7 +514,97 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit_local<CG>(drain_bar);
       mbar_wait(drain_bar, 0, nullptr, p.limit_ns, kRoleMma, &g_device_error);
     }
-  } else if (warp >= 2) {
+  } else if (LSU && warp >= 2 + kEpiWarps) {
+    // ---------------------------------------------------------------- plain loaders (every CTA)
+    // Each loader warp fills a quarter of every A and B stage, two elements
+    // per lane along the stored matrix's contiguous dimension (coalesced),
+    // then makes its shared-memory writes visible to the tensor core and
+    // arrives on the slot's full barrier (the pair leader's, with CG == 2).
+    const int lw = warp - (2 + kEpiWarps);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int k = 0; k < n_work && ok; ++k) {
+      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+      const int a_row = w.mb * kTileM + static_cast<int>(rank) * kBM;
+      const int b_col = w.nb * kTileN + static_cast<int>(rank) * Plan::kBNc;
+      for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        int got = 1;
+        if (lane == 0)
+          got = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
+                          &g_device_error);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t a_dst = smem_u32(sA + stage * Plan::kABytes);
+        const uint32_t b_dst = smem_u32(sB + stage * Plan::kBBytes);
+        const int k0 = kb * kBK;
+        const int kk2 = 2 * lane;  // this lane's pair along a 64-element row
+        // This warp's share of the stage: NA values of A and NB of B (two
+        // elements each).  All loads are issued before any store, so one
+        // memory latency covers the whole stage.
+        constexpr int NA = 32;                                       // A: 32 rows, or 16 k rows x 2
+        constexpr int NB = !BT ? 16 * (Plan::kBNc / 64) : Plan::kBNc / kLoaderWarps;
+        uint32_t va[NA], vb[NB];
+#pragma unroll
+        for (int j = 0; j < NA; ++j) {
+          if constexpr (!AT)  // A stored M x K: rows lw*32 .. +31, 64 k each
+            va[j] = load_pair(p.A, a_row + lw * 32 + j, k0 + kk2, p.lda, p.M, p.K);
+          else  // A stored K x M: k rows lw*16 .. +15, 128 m each in two passes
+            va[j] = load_pair(p.A, k0 + lw * 16 + (j & 15), a_row + (j >> 4) * 64 + kk2, p.lda,
+                              p.K, p.M);
+        }
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          if constexpr (!BT)  // B stored K x N: k rows lw*16 .. +15, kBNc columns in 64s
+            vb[j] = load_pair(p.B, k0 + lw * 16 + (j & 15), b_col + (j >> 4) * 64 + kk2, p.ldb,
+                              p.K, p.N);
+          else  // B stored N x K: n rows j*4 + lw, 64 k each
+            vb[j] = load_pair(p.B, b_col + j * kLoaderWarps + lw, k0 + kk2, p.ldb, p.N, p.K);
+        }
+#pragma unroll
+        for (int j = 0; j < NA; ++j) {
+          if constexpr (!AT)
+            st_shared_u32(a_dst + kmajor_offset(lw * 32 + j, kk2), va[j]);
+          else
+            st_shared_u32(a_dst + mnmajor_offset((j >> 4) * 64 + kk2, lw * 16 + (j & 15)), va[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          if constexpr (!BT)
+            st_shared_u32(b_dst + mnmajor_offset((j >> 4) * 64 + kk2, lw * 16 + (j & 15)), vb[j]);
+          else
+            st_shared_u32(b_dst + kmajor_offset(j * kLoaderWarps + lw, kk2), vb[j]);
+        }
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CG == 1)
+            mbar_arrive(full_bar(stage));
+          else
+            mbar_arrive_cluster(mapa_shared(full_bar(stage), 0));
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Tail: every slot released, so no commit-arrive is still on its way.
+    if (ok && lane == 0) {
+      for (int i = 0; i < STAGES; ++i) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
+                       &g_device_error))
+          break;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 2 && warp < 2 + kEpiWarps) {
     // ---------------------------------------------------------------- epilogue (every CTA)
     // Warp w drains TMEM lanes 32*(w%4) .. +31 (the lanes a warp may access),
     // 64 accumulator columns at a time, into two 4 KB boxes it owns in turn.
@@ -464,8 +623,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // piece (this lane's row, columns col0 .. col0+63).
     auto emit64 = [&](float (&va)[32], float (&vb)[32], int box_row0, int col0) {
       if constexpr (BIAS_RELU) {
-        bias_relu_32(p.bias, col0, p.N, va);
-        bias_relu_32(p.bias, col0 + 32, p.N, vb);
+        bias_relu_32(p.bias, col0, p.N, p.bias_aligned != 0, va);
+        bias_relu_32(p.bias, col0 + 32, p.N, p.bias_aligned != 0, vb);
       }
       if constexpr (OUT_F16) {
         uint32_t h[32];  // 64 fp16 values, round to nearest even
@@ -474,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           h[j] = pack_half2(va[2 * j], va[2 * j + 1]);
           h[16 + j] = pack_half2(vb[2 * j], vb[2 * j + 1]);
         }
-        if (!p.n_aligned && col0 + kBoxCols > p.N) {
+        if (p.c_plain || (!p.n_aligned && col0 + kBoxCols > p.N)) {
           store_row_tail<true>(p, box_row0 + lane, col0, h);
           return;
         }
@@ -496,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t w[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(half == 0 ? va[j] : vb[j]);
-          if (!p.n_aligned && col0 + half * kBoxCols + kBoxCols > p.N) {
+          if (p.c_plain || (!p.n_aligned && col0 + half * kBoxCols + kBoxCols > p.N)) {
             store_row_tail<false>(p, box_row0 + lane, col0 + half * kBoxCols, w);
             continue;
           }
@@ -645,19 +804,6 @@ __global__ void fill_empty_k_kernel(void *C, int64_t ldc, const __half *bias, in
       reinterpret_cast<__half *>(C)[r * ldc + c] = __float2half_rn(v);
     else
       reinterpret_cast<float *>(C)[r * ldc + c] = v;
-  }
-}
-
-// One thread waits on a barrier that nothing signals; the bounded wait gives
-// up after limit_ns, records the timeout and the kernel returns normally.
-__global__ void selftest_timeout_kernel(uint64_t limit_ns) {
-  __shared__ __align__(8) uint64_t bar;
-  __shared__ uint32_t abort_word;
-  if (threadIdx.x == 0) {
-    abort_word = 0u;
-    mbar_init(smem_u32(&bar), 1);
-    fence_mbar_init();
-    mbar_wait(smem_u32(&bar), 0, &abort_word, limit_ns, kRoleSelftest, &g_device_error);
   }
 }
 
