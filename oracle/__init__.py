@@ -16,6 +16,9 @@ Functions and the passages they follow:
   ``max(ref + bias[col], 0)`` ("domestic-GPU TileLang adoption"
   (xdnf.cn/news/333523) section 4.2).
 * ``gemm_at`` -- the same value at selected (row, col) positions.
+* ``gemm_fused`` / ``gemm_at_fused`` -- act(A.B + bias[col]) + R[row, col] with
+  act in {none, relu, gelu} ("domestic-GPU TileLang adoption" section 4.1:
+  activation and residual fused into the operator; GELU in its exact erf form).
 
 Every function is pinned by tests/test_oracle_pins.py; none is parity unpinned.
 """
@@ -55,6 +58,13 @@ def _load():
             lib.oracle_gemm_at.argtypes = [_i64, _p, _i64, _p, _i64, _p, ctypes.c_int,
                                            _p, _p, _i64, _p, ctypes.c_int]
             lib.oracle_openmp_enabled.restype = ctypes.c_int
+            lib.oracle_activation.restype = ctypes.c_double
+            lib.oracle_activation.argtypes = [ctypes.c_double, ctypes.c_int]
+            lib.oracle_gemm_fused.restype = ctypes.c_int
+            lib.oracle_gemm_fused.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, ctypes.c_int,
+                                              _p, _i64, _p, _i64, ctypes.c_int]
+            lib.oracle_gemm_at_fused.argtypes = [_i64, _p, _i64, _p, _i64, _p, ctypes.c_int, _p, _i64,
+                                                 _p, _p, _i64, _p, ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -146,6 +156,57 @@ def gemm_at(A, B, rows, cols, bias=None, relu: bool = False, threads: int | None
                            bb.ctypes.data if bb is not None else None, int(bool(relu)),
                            r.ctypes.data, c.ctypes.data, r.size, out.ctypes.data,
                            int(threads or default_threads()))
+    return out
+
+
+ACT = {"none": 0, "relu": 1, "gelu": 2}
+
+
+def activation(x: float, act: str) -> float:
+    """The oracle's activation at one point (none, relu, gelu)."""
+    return float(_load().oracle_activation(float(x), ACT[act]))
+
+
+def gemm_fused(A, B, bias=None, act: str = "none", residual=None, threads: int | None = None) -> np.ndarray:
+    """ref = act(A.B + bias[col]) + residual[row, col], float64 (the general fused epilogue)."""
+    a, b = _bits(A), _bits(B)
+    if a.ndim != 2 or b.ndim != 2 or a.shape[1] != b.shape[0]:
+        raise ValueError(f"shape mismatch {a.shape} x {b.shape}")
+    M, K = a.shape
+    N = b.shape[1]
+    bb = _bits(bias) if bias is not None else None
+    if bb is not None and bb.shape != (N,):
+        raise ValueError(f"bias must have shape ({N},)")
+    rr = _bits(residual) if residual is not None else None
+    if rr is not None and rr.shape != (M, N):
+        raise ValueError(f"residual must have shape ({M}, {N})")
+    out = np.empty((M, N), dtype=np.float64)
+    rc = _load().oracle_gemm_fused(M, N, K, a.ctypes.data, K, b.ctypes.data, N,
+                                   bb.ctypes.data if bb is not None else None, ACT[act],
+                                   rr.ctypes.data if rr is not None else None, N,
+                                   out.ctypes.data, N, int(threads or default_threads()))
+    if rc != 0:
+        raise MemoryError("oracle_gemm_fused could not allocate its decoded copy of B")
+    return out
+
+
+def gemm_at_fused(A, B, rows, cols, bias=None, act: str = "none", residual=None,
+                  threads: int | None = None) -> np.ndarray:
+    a, b = _bits(A), _bits(B)
+    M, K = a.shape
+    N = b.shape[1]
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    c = np.ascontiguousarray(np.asarray(cols, dtype=np.int64))
+    if r.size and (r.min() < 0 or r.max() >= M or c.min() < 0 or c.max() >= N):
+        raise IndexError("sample position out of range")
+    bb = _bits(bias) if bias is not None else None
+    rr = _bits(residual) if residual is not None else None
+    out = np.empty(r.shape, dtype=np.float64)
+    _load().oracle_gemm_at_fused(K, a.ctypes.data, K, b.ctypes.data, N,
+                                 bb.ctypes.data if bb is not None else None, ACT[act],
+                                 rr.ctypes.data if rr is not None else None, N,
+                                 r.ctypes.data, c.ctypes.data, r.size, out.ctypes.data,
+                                 int(threads or default_threads()))
     return out
 
 

@@ -16,7 +16,11 @@
  *     "TileLang Python DSL practice" (codechina.net/.../126997) section 3.2.
  *   - the fused epilogue, bias indexed by the output column and added before
  *     the ReLU: "domestic-GPU TileLang adoption" (xdnf.cn/news/333523)
- *     section 4.2.
+ *     section 4.2; the same page's section 4.1 names fusing an activation
+ *     and a residual connection into the GEMM, written here as
+ *     ref = act(A.B + bias[j]) + R[i][j] with act = none, ReLU or GELU.
+ *     GELU is the exact form x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)) (the
+ *     pages give no formula; this is its standard definition).
  *
  * The accumulation is fp64 (every fp16 x fp16 product is exact in fp64), so
  * the result is the exact sum up to fp64 rounding.  The k order is ascending
@@ -92,6 +96,65 @@ void oracle_f16_encode_array(const double *x, uint16_t *out, int64_t n)
         out[i] = oracle_f16_encode_rne(x[i]);
 }
 
+/* Activation codes shared by the fused routines below. */
+enum { ORACLE_ACT_NONE = 0, ORACLE_ACT_RELU = 1, ORACLE_ACT_GELU = 2 };
+
+double oracle_activation(double x, int act)
+{
+    if (act == ORACLE_ACT_RELU)
+        return x > 0.0 ? x : 0.0;
+    if (act == ORACLE_ACT_GELU)
+        return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));
+    return x;
+}
+
+/*
+ * Full product with the fused epilogue:
+ *   C[i][j] = act(sum_k A[i][k] B[k][j] + bias[j]) + R[i][j]
+ * bias (N fp16 bits) and R (M x N fp16 bits, row stride ldr) may be NULL.
+ * Returns 0, or -1 if the decoded copy of B cannot be allocated.
+ */
+int oracle_gemm_fused(int64_t M, int64_t N, int64_t K,
+                      const uint16_t *A, int64_t lda,
+                      const uint16_t *B, int64_t ldb,
+                      const uint16_t *bias, int act,
+                      const uint16_t *R, int64_t ldr,
+                      double *C, int64_t ldc, int nthreads)
+{
+    double *Bd = (double *)malloc((size_t)(K * N > 0 ? K * N : 1) * sizeof(double));
+    if (!Bd)
+        return -1;
+    for (int64_t k = 0; k < K; ++k)
+        for (int64_t j = 0; j < N; ++j)
+            Bd[k * N + j] = oracle_f16_decode(B[k * ldb + j]);
+    if (nthreads < 1)
+        nthreads = 1;
+
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t i = 0; i < M; ++i) {
+        double *c = C + i * ldc;
+        for (int64_t j = 0; j < N; ++j)
+            c[j] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double a = oracle_f16_decode(A[i * lda + k]);
+            const double *b = Bd + k * N;
+            for (int64_t j = 0; j < N; ++j)
+                c[j] += a * b[j];
+        }
+        for (int64_t j = 0; j < N; ++j) {
+            double v = c[j];
+            if (bias)
+                v += oracle_f16_decode(bias[j]);
+            v = oracle_activation(v, act);
+            if (R)
+                v += oracle_f16_decode(R[i * ldr + j]);
+            c[j] = v;
+        }
+    }
+    free(Bd);
+    return 0;
+}
+
 /*
  * Full product.  A: M x K fp16 bits, row stride lda; B: K x N, row stride ldb;
  * bias: N fp16 bits or NULL; C: M x N doubles, row stride ldc.
@@ -141,12 +204,13 @@ int oracle_gemm(int64_t M, int64_t N, int64_t K,
  * Selected outputs only: out[s] = ref[rows[s]][cols[s]], each a length-K
  * dot product in ascending k, then bias and ReLU as above.
  */
-void oracle_gemm_at(int64_t K,
-                    const uint16_t *A, int64_t lda,
-                    const uint16_t *B, int64_t ldb,
-                    const uint16_t *bias, int relu,
-                    const int64_t *rows, const int64_t *cols, int64_t count,
-                    double *out, int nthreads)
+void oracle_gemm_at_fused(int64_t K,
+                          const uint16_t *A, int64_t lda,
+                          const uint16_t *B, int64_t ldb,
+                          const uint16_t *bias, int act,
+                          const uint16_t *R, int64_t ldr,
+                          const int64_t *rows, const int64_t *cols, int64_t count,
+                          double *out, int nthreads)
 {
     if (nthreads < 1)
         nthreads = 1;
@@ -158,10 +222,22 @@ void oracle_gemm_at(int64_t K,
             acc += oracle_f16_decode(A[i * lda + k]) * oracle_f16_decode(B[k * ldb + j]);
         if (bias)
             acc += oracle_f16_decode(bias[j]);
-        if (relu)
-            acc = acc > 0.0 ? acc : 0.0;
+        acc = oracle_activation(acc, act);
+        if (R)
+            acc += oracle_f16_decode(R[i * ldr + j]);
         out[s] = acc;
     }
+}
+
+void oracle_gemm_at(int64_t K,
+                    const uint16_t *A, int64_t lda,
+                    const uint16_t *B, int64_t ldb,
+                    const uint16_t *bias, int relu,
+                    const int64_t *rows, const int64_t *cols, int64_t count,
+                    double *out, int nthreads)
+{
+    oracle_gemm_at_fused(K, A, lda, B, ldb, bias, relu ? ORACLE_ACT_RELU : ORACLE_ACT_NONE,
+                         NULL, 0, rows, cols, count, out, nthreads);
 }
 
 int oracle_openmp_enabled(void)

@@ -44,6 +44,10 @@ def read_golden_blocks(name):
                 blocks.append(cur)
             elif key == "shape":
                 cur["shape"] = tuple(int(v) for v in vals)
+            elif key == "act":
+                cur["act"] = vals[0]
+            elif vals == ["none"]:
+                cur[key] = None
             else:
                 cur[key] = [float(v) for v in vals]
     return blocks

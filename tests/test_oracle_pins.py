@@ -332,3 +332,205 @@ def test_planted_mistake_is_caught(mutant):
         except (AssertionError, ValueError, IndexError):
             failed.append(pin.__name__)
     assert failed, f"{mutant.__name__} passed every pin"
+
+
+# ----------------------------------------------------------------------------- the general fused epilogue
+# ref = act(A.B + bias[col]) + R[row, col], act in {none, relu, gelu}
+# ("domestic-GPU TileLang adoption" section 4.1: activation and residual fused
+# into the GEMM; section 4.2: bias by output column, before the activation).
+# GELU is x * Phi(x), Phi the standard normal CDF, checked against scipy's
+# normal CDF and against the symmetry gelu(x) - gelu(-x) = x.
+
+from scipy.special import ndtr  # noqa: E402
+
+PHI_1 = 0.841344746068542948  # the standard normal CDF at 1 (table value)
+
+
+def _gelu_scipy(x):
+    x = np.asarray(x, dtype=np.float64)
+    return x * ndtr(x)
+
+
+def fpin_golden(g):
+    for ex in read_golden_blocks("fused_epilogue_worked_examples.txt"):
+        M, N, K = ex["shape"]
+        A = f16(ex["A"]).reshape(M, K)
+        B = f16(ex["B"]).reshape(K, N)
+        bias = None if ex["bias"] is None else f16(ex["bias"])
+        R = None if ex["R"] is None else f16(ex["R"]).reshape(M, N)
+        C = np.array(ex["C"]).reshape(M, N)
+        got = g(A, B, bias, ex["act"], R)
+        assert np.all(np.abs(got - C) <= 1e-15), (ex["name"], got, C)
+
+
+def fpin_gelu_library(g):
+    # A = I (K = N), B = x as fp16: the output row is act(x) exactly at the input points.
+    x = np.concatenate([np.linspace(-6, 6, 61), [-1.0, 1.0, 0.0, 1e-4, -1e-4, 0.5, -0.5]])
+    xb = f16(x)
+    n = xb.size
+    out = g(np.ones((1, 1), np.float16), xb.reshape(1, n), None, "gelu", None)[0]
+    want = _gelu_scipy(dec(xb))
+    assert np.all(np.abs(out - want) <= 4e-15 * (1 + np.abs(dec(xb)))), np.max(np.abs(out - want))
+
+
+def fpin_gelu_symmetry_and_limits(g):
+    xb = f16(np.linspace(0, 8, 33))
+    pos = g(np.ones((1, 1), np.float16), xb.reshape(1, -1), None, "gelu", None)[0]
+    neg = g(-np.ones((1, 1), np.float16), xb.reshape(1, -1), None, "gelu", None)[0]
+    x = dec(xb)
+    assert np.all(np.abs((pos - neg) - x) <= 1e-14 * (1 + x))
+    assert pos[0] == 0.0 and neg[0] == 0.0
+    assert abs(pos[-1] - 8.0) < 1e-13 and abs(neg[-1]) < 1e-13
+    one = g(np.ones((1, 1), np.float16), np.ones((1, 1), np.float16), None, "gelu", None)[0, 0]
+    assert abs(one - PHI_1) <= 1e-15
+
+
+def fpin_residual_is_added_after_activation(g):
+    rng = np.random.default_rng(6)
+    M, N, K = 5, 7, 3
+    A = f16(rng.uniform(-1, 1, (M, K)))
+    B = f16(rng.uniform(-1, 1, (K, N)))
+    bias = f16(rng.uniform(-0.5, 0.5, N))
+    R = f16(rng.uniform(-2, 2, (M, N)))
+    for act in ("none", "relu", "gelu"):
+        with_r = g(A, B, bias, act, R)
+        without = g(A, B, bias, act, None)
+        assert np.array_equal(with_r, without + dec(R)), act
+    # a zero product leaves act(bias) + R: the residual keeps its row and column
+    zero = g(np.zeros((M, K), np.float16), B, bias, "relu", R)
+    assert np.array_equal(zero, np.maximum(dec(bias), 0.0)[None, :] + dec(R))
+
+
+def fpin_fused_reduces_to_bias_relu(g):
+    rng = np.random.default_rng(7)
+    M, N, K = 9, 12, 70
+    A = f16(rng.uniform(-1, 1, (M, K)))
+    B = f16(rng.uniform(-1, 1, (K, N)))
+    bias = f16(rng.uniform(-0.5, 0.5, N))
+    want = dec(A) @ dec(B) + dec(bias)[None, :]
+    scale = np.abs(dec(A)) @ np.abs(dec(B)) + np.abs(dec(bias))[None, :]
+    got = g(A, B, bias, "relu", None)
+    assert np.all(np.abs(got - np.maximum(want, 0.0)) <= 1e-12 * scale)
+    got = g(A, B, None, "none", None)
+    assert np.all(np.abs(got - dec(A) @ dec(B)) <= 1e-12 * scale)
+
+
+FPINS = [fpin_golden, fpin_gelu_library, fpin_gelu_symmetry_and_limits,
+         fpin_residual_is_added_after_activation, fpin_fused_reduces_to_bias_relu]
+
+
+def oracle_fused(A, B, bias, act, R):
+    return oracle.gemm_fused(A, B, bias=bias, act=act, residual=R, threads=2)
+
+
+@pytest.mark.parametrize("pin", FPINS, ids=lambda p: p.__name__)
+def test_oracle_fused_pins(pin):
+    pin(oracle_fused)
+
+
+def test_fused_sampled_equals_full_bit_for_bit():
+    rng = np.random.default_rng(8)
+    M, N, K = 40, 33, 129
+    A = f16(rng.uniform(-1, 1, (M, K)))
+    B = f16(rng.uniform(-1, 1, (K, N)))
+    bias = f16(rng.uniform(-0.5, 0.5, N))
+    R = f16(rng.uniform(-1, 1, (M, N)))
+    rows = rng.integers(0, M, 200)
+    cols = rng.integers(0, N, 200)
+    for act in ("none", "relu", "gelu"):
+        full = oracle.gemm_fused(A, B, bias=bias, act=act, residual=R, threads=3)
+        at = oracle.gemm_at_fused(A, B, rows, cols, bias=bias, act=act, residual=R, threads=2)
+        assert np.array_equal(at, full[rows, cols]), act
+    assert np.array_equal(oracle.gemm_fused(A, B, bias=bias, act="relu", threads=2),
+                          oracle.gemm(A, B, bias=bias, relu=True, threads=2))
+
+
+def test_oracle_activation_points():
+    assert oracle.activation(-2.0, "relu") == 0.0 and oracle.activation(3.0, "relu") == 3.0
+    assert oracle.activation(-2.5, "none") == -2.5
+    assert abs(oracle.activation(1.0, "gelu") - PHI_1) <= 1e-15
+
+
+def _fref(A, B, bias, act, R):
+    C = dec(A) @ dec(B)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    if act == "relu":
+        C = np.maximum(C, 0.0)
+    elif act == "gelu":
+        C = _gelu_scipy(C)
+    if R is not None:
+        C = C + dec(R)
+    return C
+
+
+def fmutant_residual_inside_activation(A, B, bias, act, R):
+    C = dec(A) @ dec(B)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    if R is not None:
+        C = C + dec(R)
+    return _fref(np.ones((C.shape[0], 1), np.float16), np.zeros((1, C.shape[1]), np.float16),
+                 None, "none", None) + (np.maximum(C, 0.0) if act == "relu" else
+                                        _gelu_scipy(C) if act == "gelu" else C)
+
+
+def fmutant_gelu_tanh_form(A, B, bias, act, R):
+    C = dec(A) @ dec(B)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    if act == "relu":
+        C = np.maximum(C, 0.0)
+    elif act == "gelu":
+        C = 0.5 * C * (1 + np.tanh(math.sqrt(2 / math.pi) * (C + 0.044715 * C ** 3)))
+    return C + (dec(R) if R is not None else 0.0)
+
+
+def fmutant_gelu_sign(A, B, bias, act, R):
+    C = dec(A) @ dec(B)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    if act == "relu":
+        C = np.maximum(C, 0.0)
+    elif act == "gelu":
+        C = C * ndtr(-C)
+    return C + (dec(R) if R is not None else 0.0)
+
+
+def fmutant_residual_transposed(A, B, bias, act, R):
+    C = _fref(A, B, bias, act, None)
+    if R is not None:
+        M, N = C.shape
+        C = C + dec(R).reshape(N, M).T
+    return C
+
+
+def fmutant_residual_dropped(A, B, bias, act, R):
+    return _fref(A, B, bias, act, None)
+
+
+def fmutant_residual_shifted_row(A, B, bias, act, R):
+    C = _fref(A, B, bias, act, None)
+    if R is not None:
+        C = C + np.roll(dec(R), 1, axis=0)
+    return C
+
+
+FMUTANTS = [fmutant_residual_inside_activation, fmutant_gelu_tanh_form, fmutant_gelu_sign,
+            fmutant_residual_transposed, fmutant_residual_dropped, fmutant_residual_shifted_row]
+
+
+def test_fused_numpy_copy_passes_pins():
+    for pin in FPINS:
+        pin(_fref)
+
+
+@pytest.mark.parametrize("mutant", FMUTANTS, ids=lambda m: m.__name__)
+def test_fused_planted_mistake_is_caught(mutant):
+    failed = []
+    for pin in FPINS:
+        try:
+            pin(mutant)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"{mutant.__name__} passed every pin"
