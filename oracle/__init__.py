@@ -104,6 +104,28 @@ def f16_decode(bits) -> np.ndarray:
     return out
 
 
+def _values(x) -> np.ndarray:
+    """A residual in the output's type as exact float64 values: fp16 through the
+    oracle's own decoder, fp32 (and fp64) by numpy's exact widening."""
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            if x.dtype == torch.float16:
+                return f16_decode(x)
+            if x.dtype not in (torch.float32, torch.float64):
+                raise TypeError(f"residual must be fp16 or fp32, got {x.dtype}")
+            x = x.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.asarray(x)
+    if x.dtype in (np.float16, np.uint16, np.int16):
+        return f16_decode(x)
+    if x.dtype not in (np.float32, np.float64):
+        raise TypeError(f"residual must be fp16 or fp32, got {x.dtype}")
+    return np.ascontiguousarray(x.astype(np.float64))
+
+
 def f16_encode_rne(x) -> np.ndarray:
     """Round float64 values to binary16 (ties to even); returns the uint16 bit patterns."""
     x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
@@ -168,7 +190,8 @@ def activation(x: float, act: str) -> float:
 
 
 def gemm_fused(A, B, bias=None, act: str = "none", residual=None, threads: int | None = None) -> np.ndarray:
-    """ref = act(A.B + bias[col]) + residual[row, col], float64 (the general fused epilogue)."""
+    """ref = act(A.B + bias[col]) + residual[row, col], float64 (the general fused epilogue).
+    The residual has the output's type: fp16 (decoded here) or fp32."""
     a, b = _bits(A), _bits(B)
     if a.ndim != 2 or b.ndim != 2 or a.shape[1] != b.shape[0]:
         raise ValueError(f"shape mismatch {a.shape} x {b.shape}")
@@ -177,7 +200,7 @@ def gemm_fused(A, B, bias=None, act: str = "none", residual=None, threads: int |
     bb = _bits(bias) if bias is not None else None
     if bb is not None and bb.shape != (N,):
         raise ValueError(f"bias must have shape ({N},)")
-    rr = _bits(residual) if residual is not None else None
+    rr = _values(residual) if residual is not None else None
     if rr is not None and rr.shape != (M, N):
         raise ValueError(f"residual must have shape ({M}, {N})")
     out = np.empty((M, N), dtype=np.float64)
@@ -200,7 +223,9 @@ def gemm_at_fused(A, B, rows, cols, bias=None, act: str = "none", residual=None,
     if r.size and (r.min() < 0 or r.max() >= M or c.min() < 0 or c.max() >= N):
         raise IndexError("sample position out of range")
     bb = _bits(bias) if bias is not None else None
-    rr = _bits(residual) if residual is not None else None
+    rr = _values(residual) if residual is not None else None
+    if rr is not None and rr.shape != (M, N):
+        raise ValueError(f"residual must have shape ({M}, {N})")
     out = np.empty(r.shape, dtype=np.float64)
     _load().oracle_gemm_at_fused(K, a.ctypes.data, K, b.ctypes.data, N,
                                  bb.ctypes.data if bb is not None else None, ACT[act],

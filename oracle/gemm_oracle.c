@@ -111,14 +111,16 @@ double oracle_activation(double x, int act)
 /*
  * Full product with the fused epilogue:
  *   C[i][j] = act(sum_k A[i][k] B[k][j] + bias[j]) + R[i][j]
- * bias (N fp16 bits) and R (M x N fp16 bits, row stride ldr) may be NULL.
+ * bias (N fp16 bits) may be NULL.  R holds the residual's values (M x N
+ * doubles, row stride ldr: the residual has the output's type, fp16 or fp32,
+ * and either converts to fp64 exactly) and may be NULL.
  * Returns 0, or -1 if the decoded copy of B cannot be allocated.
  */
 int oracle_gemm_fused(int64_t M, int64_t N, int64_t K,
                       const uint16_t *A, int64_t lda,
                       const uint16_t *B, int64_t ldb,
                       const uint16_t *bias, int act,
-                      const uint16_t *R, int64_t ldr,
+                      const double *R, int64_t ldr,
                       double *C, int64_t ldc, int nthreads)
 {
     double *Bd = (double *)malloc((size_t)(K * N > 0 ? K * N : 1) * sizeof(double));
@@ -147,7 +149,7 @@ int oracle_gemm_fused(int64_t M, int64_t N, int64_t K,
                 v += oracle_f16_decode(bias[j]);
             v = oracle_activation(v, act);
             if (R)
-                v += oracle_f16_decode(R[i * ldr + j]);
+                v += R[i * ldr + j];
             c[j] = v;
         }
     }
@@ -202,13 +204,13 @@ int oracle_gemm(int64_t M, int64_t N, int64_t K,
 
 /*
  * Selected outputs only: out[s] = ref[rows[s]][cols[s]], each a length-K
- * dot product in ascending k, then bias and ReLU as above.
+ * dot product in ascending k, then bias, activation and residual as above.
  */
 void oracle_gemm_at_fused(int64_t K,
                           const uint16_t *A, int64_t lda,
                           const uint16_t *B, int64_t ldb,
                           const uint16_t *bias, int act,
-                          const uint16_t *R, int64_t ldr,
+                          const double *R, int64_t ldr,
                           const int64_t *rows, const int64_t *cols, int64_t count,
                           double *out, int nthreads)
 {
@@ -224,7 +226,7 @@ void oracle_gemm_at_fused(int64_t K,
             acc += oracle_f16_decode(bias[j]);
         acc = oracle_activation(acc, act);
         if (R)
-            acc += oracle_f16_decode(R[i * ldr + j]);
+            acc += R[i * ldr + j];
         out[s] = acc;
     }
 }

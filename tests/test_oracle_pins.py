@@ -534,3 +534,17 @@ def test_fused_planted_mistake_is_caught(mutant):
         except (AssertionError, ValueError, IndexError):
             failed.append(pin.__name__)
     assert failed, f"{mutant.__name__} passed every pin"
+
+
+def test_fused_residual_in_fp32():
+    # An fp32 residual enters at its exact value: R = 2^-20 * odd integers,
+    # which fp16 cannot hold, is added exactly after the activation.
+    rng = np.random.default_rng(9)
+    M, N, K = 4, 6, 5
+    A = f16(rng.uniform(-1, 1, (M, K)))
+    B = f16(rng.uniform(-1, 1, (K, N)))
+    R = (rng.integers(-2 ** 19, 2 ** 19, (M, N)) * 2 + 1).astype(np.float32) * np.float32(2.0 ** -20)
+    base = oracle.gemm_fused(A, B, act="gelu", threads=1)
+    got = oracle.gemm_fused(A, B, act="gelu", residual=R, threads=1)
+    assert np.array_equal(got, base + R.astype(np.float64))
+    assert not np.array_equal(got, base + dec(R.astype(np.float16)))
