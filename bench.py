@@ -210,18 +210,35 @@ def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float)
     return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
-def cpu_oracle_rate(w: wl.Workload, target_s: float, threads: int, A=None, B=None, bias=None):
-    """Time the oracle on a row sample of the workload sized for about target_s seconds.
-    Returns (TFLOP/s, rows timed, seconds)."""
+def all_workloads():
+    return {**wl.WORKLOADS, **wl.EPILOGUE_WORKLOADS}
+
+
+def workload_residual(w: wl.Workload, seed: int = 0):
+    return wl.make_residual(w.M, w.N, w.out, seed) if w.residual else None
+
+
+def oracle_rows(w: wl.Workload, A, B, bias, R, rows: int, threads: int):
+    """The oracle's result for the first `rows` output rows of the workload."""
     import oracle
 
+    if w.act is not None:
+        return oracle.gemm_fused(A[:rows], B, bias=bias, act=w.act,
+                                 residual=R[:rows] if R is not None else None, threads=threads)
+    return oracle.gemm(A[:rows], B, bias=bias, relu=w.bias_relu, threads=threads)
+
+
+def cpu_oracle_rate(w: wl.Workload, target_s: float, threads: int, A=None, B=None, bias=None, R=None):
+    """Time the oracle on a row sample of the workload sized for about target_s seconds.
+    Returns (TFLOP/s, rows timed, seconds)."""
     if A is None:
         A, B, bias = wl.workload_operands(w)
+        R = workload_residual(w)
     # grow a row sample until it takes a tenth of the target, then scale to the target
     probe = max(1, min(w.M, threads))
     while True:
         t0 = time.perf_counter()
-        oracle.gemm(A[:probe], B, bias=bias, relu=w.bias_relu, threads=threads)
+        oracle_rows(w, A, B, bias, R, probe, threads)
         dt = max(time.perf_counter() - t0, 1e-6)
         if dt >= target_s / 10 or probe >= w.M:
             break
@@ -229,7 +246,7 @@ def cpu_oracle_rate(w: wl.Workload, target_s: float, threads: int, A=None, B=Non
     rows = int(min(w.M, max(probe, probe * target_s / dt)))
     rows = max(1, (rows // threads) * threads) if rows >= threads else rows
     t0 = time.perf_counter()
-    oracle.gemm(A[:rows], B, bias=bias, relu=w.bias_relu, threads=threads)
+    oracle_rows(w, A, B, bias, R, rows, threads)
     dt = time.perf_counter() - t0
     return 2.0 * rows * w.N * w.K / dt / 1e12, rows, dt
 
@@ -242,13 +259,14 @@ def run_reference(args, w: wl.Workload):
 
     threads = oracle.default_threads()
     A, B, bias = wl.workload_operands(w)
+    R = workload_residual(w)
     # each step: a row sample sized so that warmup + steps stay within a few minutes
     per_step = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
-    _, rows, _ = cpu_oracle_rate(w, per_step, threads, A, B, bias)
+    _, rows, _ = cpu_oracle_rate(w, per_step, threads, A, B, bias, R)
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        oracle.gemm(A[:rows], B, bias=bias, relu=w.bias_relu, threads=threads)
+        oracle_rows(w, A, B, bias, R, rows, threads)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     flops = 2.0 * rows * w.N * w.K
@@ -268,8 +286,11 @@ def run_reference(args, w: wl.Workload):
 
 
 def workload_config(w: wl.Workload, kcfg):
+    epi = "bias_relu" if w.bias_relu else "none"
+    if w.act is not None:
+        epi = f"bias_{w.act}" + ("_residual (separate fp16 R, read once)" if w.residual else "")
     return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": w.out,
-            "epilogue": "bias_relu" if w.bias_relu else "none", "accumulate": "f32",
+            "epilogue": epi, "accumulate": "f32",
             "inputs": "uniform[-1,1] fp16" if w.dist == "uniform" else "normal(0,1)*0.25 fp16",
             "l2": f"flushed before every step ({FLUSH_BYTES >> 20} MiB write, untimed)",
             "kernel_config": kcfg, "parallelism": "independent problem per GPU"}
@@ -280,7 +301,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=wl.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=wl.WORKLOAD_ORDER + list(wl.EPILOGUE_WORKLOADS))
     ap.add_argument("--impl", default="tlg", choices=["tlg", "reference"])
     ap.add_argument("--config", default=None, help="JSON tlg_config override (tuning sweeps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -293,7 +315,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
-    w = wl.WORKLOADS[args.workload]
+    w = all_workloads()[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -305,6 +327,7 @@ def main(argv=None):
     dev = torch.device("cuda", local if world > 1 else 0)
     stream = torch.cuda.current_stream(dev)
     A, B, bias = wl.workload_operands(w, seed=rank)
+    R = workload_residual(w, seed=rank)
     at, bt = args.layout[0] == "T", args.layout[1] == "T"
     if at:
         A = A.t().contiguous()  # stored K x M; the product uses its transpose
@@ -321,22 +344,31 @@ def main(argv=None):
 
     dA, dB = padded(A, args.ld_pad), padded(B, args.ld_pad)
     dbias = bias.to(dev) if bias is not None else None
+    dR = padded(R, args.ld_pad) if R is not None else None
     dC = padded(torch.empty((w.M, w.N), dtype=torch.float32 if w.out == "f32" else torch.float16),
                 args.ld_pad)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     override = json.loads(args.config) if args.config else None
-    kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu, request=override)
+    kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.has_bias, request=override)
     # The split-K tail needs caller scratch; allocated once here, outside the timed region.
-    ws_bytes = tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, w.out, w.bias_relu, override)
+    ws_bytes = tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, w.out, w.has_bias, override)
     ws = tlg.tlg_workspace(ws_bytes, device=dev) if ws_bytes > 0 else None
-    plain_name = ("tlg_gemm_bias_relu_f16" if w.bias_relu else
+    fused = w.act is not None
+    plain_name = ("tlg_gemm_fused" if fused else "tlg_gemm_bias_relu_f16" if w.bias_relu else
                   ("tlg_gemm_f16f16" if w.out == "f16" else "tlg_gemm_f16f32"))
-    use_op = at or bt or args.ld_pad != 0
-    use_ex = (ws is not None or override is not None) and not use_op
+    use_op = (at or bt or args.ld_pad != 0) and not fused
+    use_ex = (ws is not None or override is not None) and not use_op and not fused
     entry = "tlg_gemm_op" if use_op else ("tlg_gemm_ex" if use_ex else plain_name)
 
+    def fused_step(config=None, workspace=None):
+        tlg.tlg_gemm_fused(dA, dB, args.layout[0], args.layout[1], bias=dbias, activation=w.act,
+                           residual=dR, C=dC, out=w.out, config=config, workspace=workspace,
+                           stream=stream)
+
     def plain_step():
-        if w.bias_relu:
+        if fused:
+            fused_step()
+        elif w.bias_relu:
             tlg.tlg_gemm_bias_relu_f16(dA, dB, dbias, dC, stream=stream)
         elif w.out == "f16":
             tlg.tlg_gemm_f16f16(dA, dB, dC, stream=stream)
@@ -344,7 +376,9 @@ def main(argv=None):
             tlg.tlg_gemm_f16f32(dA, dB, dC, stream=stream)
 
     def step():
-        if use_op:
+        if fused:
+            fused_step(override, ws)
+        elif use_op:
             tlg.tlg_gemm_op(dA, dB, args.layout[0], args.layout[1], dbias, dC, out=w.out, config=override,
                             workspace=ws, stream=stream)
         elif use_ex:
@@ -386,7 +420,7 @@ def main(argv=None):
 
     # The same steps through the plain entry point (no workspace), for comparison.
     plain = None
-    if use_ex and override is None and not use_op:
+    if use_ex and override is None and not use_op and not fused:
         for _ in range(args.warmup):
             flush.fill_(1.0)
             plain_step()
@@ -407,8 +441,10 @@ def main(argv=None):
     if not args.no_e2e:
         hA, hB = A.pin_memory(), B.pin_memory()
         hbias = bias.pin_memory() if bias is not None else None
+        hR = R.pin_memory() if R is not None else None
         hC = torch.empty(dC.shape, dtype=dC.dtype).pin_memory()
         h2d = hA.numel() * 2 + hB.numel() * 2 + (hbias.numel() * 2 if hbias is not None else 0)
+        h2d += hR.numel() * hR.element_size() if hR is not None else 0
         d2h = hC.numel() * hC.element_size()
 
         def e2e_step():
@@ -416,6 +452,8 @@ def main(argv=None):
             dB.copy_(hB, non_blocking=True)
             if hbias is not None:
                 dbias.copy_(hbias, non_blocking=True)
+            if hR is not None:
+                dR.copy_(hR, non_blocking=True)
             step()
             hC.copy_(dC, non_blocking=True)
 
@@ -459,7 +497,7 @@ def main(argv=None):
         import oracle
 
         threads = oracle.default_threads()
-        rate, rows, secs = cpu_oracle_rate(w, 10.0, threads, A, B, bias)
+        rate, rows, secs = cpu_oracle_rate(w, 10.0, threads, A, B, bias, R)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{rows} of {w.M} output rows (all N={w.N} columns, K={w.K}) in {secs:.1f} s, fp64"}
 

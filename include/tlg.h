@@ -13,7 +13,8 @@
  * "TileLang Python DSL practice", codechina.net/.../126997, section 3.2: the
  * same product written to an fp32 C).  The fused variant applies a per-column
  * bias and a ReLU before the fp16 store ("domestic-GPU TileLang adoption",
- * xdnf.cn/news/333523, section 4.2).
+ * xdnf.cn/news/333523, section 4.2); tlg_gemm_fused generalises it to a bias,
+ * an activation (ReLU or GELU) and a residual connection (same page, 4.1).
  *
  * Conventions shared by every entry point below:
  *
@@ -37,7 +38,8 @@
  *  - Sizes: 0 <= M, N, K <= 2^31 - 257, and ceil(M/128)*ceil(N/64) below 2^31
  *    (larger sizes give TLG_ERR_UNSUPPORTED); lda >= K, ldb >= N, ldc >= N.
  *    M == 0 or N == 0: nothing is written, TLG_OK.  K == 0: the empty sum is
- *    0, so C = 0 (bias variant: C = fp16(max(bias[col], 0))).
+ *    0, so C = 0 (bias variant: C = fp16(max(bias[col], 0)); tlg_gemm_fused:
+ *    C = act(bias[col]) + residual).
  *  - The return value is the only error channel; nothing throws or aborts.
  *    Errors found before launch leave C untouched.  An error of the launch
  *    itself is TLG_ERR_CUDA.  Errors the kernel detects on the device (a
@@ -232,9 +234,63 @@ tlg_status tlg_gemm_op(int64_t M, int64_t N, int64_t K,
                        void *workspace, size_t workspace_bytes,
                        void *stream);
 
+/* Activations of the fused epilogue. */
+typedef enum tlg_activation {
+    TLG_ACT_NONE = 0,
+    TLG_ACT_RELU = 1, /* max(x, 0) */
+    TLG_ACT_GELU = 2  /* x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)), the exact (erf) form */
+} tlg_activation;
+
+/*
+ * The general fused epilogue of tlg_gemm_fused:
+ *
+ *   C[i][j] = act(acc[i][j] + bias[j]) + residual[i][j]
+ *
+ * acc is the fp32 accumulator of op(A) . op(B); everything is computed in
+ * fp32 and rounded once to C's type at the store.
+ *   bias       : N fp16 values (device memory), or NULL for none
+ *   activation : a tlg_activation
+ *   residual   : M x N row-major in C's type (fp16 for TLG_OUT_F16, fp32 for
+ *                TLG_OUT_F32), row stride ldr >= N elements, device memory;
+ *                or NULL for none.  It may be C itself (residual == C and
+ *                ldr == ldc: an in-place residual connection); any other
+ *                overlap with C is TLG_ERR_INVALID_ARG.
+ * Page: "domestic-GPU TileLang adoption" (xdnf.cn/news/333523) section 4.1
+ * names fusing an activation and a residual connection into the GEMM;
+ * section 4.2 gives the bias-by-column-then-ReLU form (bias, TLG_ACT_RELU,
+ * no residual, fp16 C is exactly tlg_gemm_bias_relu_f16).  The pages print
+ * no GELU formula; the exact erf form is used.
+ */
+typedef struct tlg_fused_epilogue {
+    const void *bias;
+    int32_t activation;
+    const void *residual;
+    int64_t ldr;
+} tlg_fused_epilogue;
+
+/*
+ * C = act(op(A) . op(B) + bias) + residual, with either output type.
+ * Operands, op_a / op_b, configuration, workspace and errors as tlg_gemm_op.
+ * epilogue == NULL, or one with no bias, TLG_ACT_NONE and no residual, is
+ * the plain product.  An activation outside tlg_activation is
+ * TLG_ERR_INVALID_ARG; a residual pointer not aligned to its element is
+ * TLG_ERR_ALIGNMENT (a 16-byte aligned base and row stride let it be read
+ * 16 bytes at a time).  K == 0 gives C = act(bias) + residual.
+ */
+tlg_status tlg_gemm_fused(int64_t M, int64_t N, int64_t K,
+                          tlg_op op_a, const void *A, int64_t lda,
+                          tlg_op op_b, const void *B, int64_t ldb,
+                          const tlg_fused_epilogue *epilogue,
+                          void *C, int64_t ldc, tlg_out out,
+                          const tlg_config *config,
+                          void *workspace, size_t workspace_bytes,
+                          void *stream);
+
 /*
  * Workspace bytes tlg_gemm_ex would use for this shape and configuration
  * (NULL = automatic) when given enough; 0 when every tile runs whole.
+ * The answer does not depend on the epilogue, so it also holds for
+ * tlg_gemm_op and tlg_gemm_fused.
  * No kernel is launched; the only CUDA calls read device attributes.
  */
 tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,

@@ -94,3 +94,32 @@ def test_binding_validates_shapes(lib_path):
         tlg.tlg_gemm_f16f32(A.float(), torch.zeros((8, 8), dtype=torch.float16))
     with pytest.raises(ValueError):
         tlg.tlg_gemm_f16f32(torch.zeros((8, 4), dtype=torch.float16).t(), torch.zeros((8, 8), dtype=torch.float16))
+
+
+def test_fused_epilogue_host_side_rejections(lib_path):
+    import tiled_dense_gemm_tlg_b200 as tlg
+    lib = tlg.raw_library()
+    A = 1 << 20
+    C = A * 2
+
+    def call(epi, out=1, c=C, ldc=8):
+        return lib.tlg_gemm_fused(8, 8, 8, 0, A, 8, 0, A, 8, ctypes.byref(epi) if epi is not None else None,
+                                  c, ldc, out, None, None, 0, None)
+
+    E = tlg.tlg_fused_epilogue
+    assert call(E(None, 3, None, 0)) == tlg.TLG_ERR_INVALID_ARG          # no such activation
+    assert call(E(None, -1, None, 0)) == tlg.TLG_ERR_INVALID_ARG
+    assert call(E(None, 2, C + 64, 8)) == tlg.TLG_ERR_INVALID_ARG        # residual overlaps C, shifted
+    assert call(E(None, 2, C, 16)) == tlg.TLG_ERR_INVALID_ARG            # same base, other stride
+    assert call(E(None, 0, A * 3, 7)) == tlg.TLG_ERR_INVALID_ARG         # ldr < N
+    assert call(E(None, 0, A * 3 + 1, 8)) == tlg.TLG_ERR_ALIGNMENT       # fp16 residual on an odd address
+    assert call(E(None, 0, A * 3 + 2, 8), out=0) == tlg.TLG_ERR_ALIGNMENT  # fp32 residual needs 4 bytes
+    assert call(E(A + 1, 0, None, 0)) == tlg.TLG_ERR_ALIGNMENT           # bias on an odd address
+    assert lib.tlg_gemm_fused(8, 8, 8, 2, A, 8, 0, A, 8, None, C, 8, 1, None, None, 0, None) == tlg.TLG_ERR_INVALID_ARG
+    assert lib.tlg_gemm_fused(8, 8, 8, 0, A, 8, 0, A, 8, None, C, 8, 5, None, None, 0, None) == tlg.TLG_ERR_INVALID_ARG
+    # residual must not overlap a split-K workspace either
+    assert lib.tlg_gemm_fused(8, 8, 8, 0, A, 8, 0, A, 8, ctypes.byref(E(None, 0, A * 4, 8)), C, 8, 1, None,
+                              A * 4, 4096, None) == tlg.TLG_ERR_INVALID_ARG
+    # empty shapes are fine with any valid descriptor
+    assert lib.tlg_gemm_fused(0, 8, 8, 0, None, 8, 0, None, 8, ctypes.byref(E(None, 2, None, 0)), None, 8, 1,
+                              None, None, 0, None) == tlg.TLG_OK

@@ -13,6 +13,8 @@ Functions (same names as the C entry points):
 * ``tlg_gemm_f16f16(A, B, C=None)``        C fp16 = A.B
 * ``tlg_gemm_bias_relu_f16(A, B, bias, C=None)``  C fp16 = max(A.B + bias, 0)
 * ``tlg_gemm_ex(...)``                     any of the above with an explicit configuration
+* ``tlg_gemm_op(...)``                     operands stored transposed
+* ``tlg_gemm_fused(...)``                  C = act(op(A).op(B) + bias) + residual
 * ``tlg_choose_config``, ``tlg_device_error``, ``tlg_selftest_timeout``,
   ``tlg_status_string``, ``tlg_version``
 
@@ -41,9 +43,11 @@ TLG_OK, TLG_ERR_INVALID_ARG, TLG_ERR_ALIGNMENT, TLG_ERR_UNSUPPORTED, TLG_ERR_CUD
 TLG_OUT_F32, TLG_OUT_F16 = 0, 1
 TLG_EPI_NONE, TLG_EPI_BIAS_RELU = 0, 1
 TLG_OP_N, TLG_OP_T = 0, 1
+TLG_ACT_NONE, TLG_ACT_RELU, TLG_ACT_GELU = 0, 1, 2
+_ACT = {"none": TLG_ACT_NONE, "relu": TLG_ACT_RELU, "gelu": TLG_ACT_GELU}
 
 EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-            "tlg_gemm_op", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
+            "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
             "tlg_version")
 
 
@@ -56,6 +60,11 @@ class tlg_config(ctypes.Structure):
         return {f: getattr(self, f) for f, _ in self._fields_}
 
 
+class tlg_fused_epilogue(ctypes.Structure):
+    _fields_ = [("bias", ctypes.c_void_p), ("activation", ctypes.c_int32),
+                ("residual", ctypes.c_void_p), ("ldr", ctypes.c_int64)]
+
+
 _i64, _p, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
 _lib.tlg_gemm_f16f32.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p]
 _lib.tlg_gemm_f16f16.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p]
@@ -65,6 +74,9 @@ _lib.tlg_gemm_ex.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64,
                              ctypes.POINTER(tlg_config), _p, _sz, _p]
 _lib.tlg_gemm_op.argtypes = [_i64, _i64, _i64, _i32, _p, _i64, _i32, _p, _i64, _p, _p, _i64, _i32, _i32,
                              ctypes.POINTER(tlg_config), _p, _sz, _p]
+_lib.tlg_gemm_fused.argtypes = [_i64, _i64, _i64, _i32, _p, _i64, _i32, _p, _i64,
+                                ctypes.POINTER(tlg_fused_epilogue), _p, _i64, _i32,
+                                ctypes.POINTER(tlg_config), _p, _sz, _p]
 _lib.tlg_gemm_ex_noalloc.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i32, _i32,
                                      ctypes.POINTER(tlg_config), _p]
 _lib.tlg_gemm_workspace_size.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config),
@@ -76,7 +88,7 @@ _lib.tlg_status_string.argtypes = [_i32]
 _lib.tlg_status_string.restype = ctypes.c_char_p
 _lib.tlg_version.restype = ctypes.c_int32
 for _name in ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-              "tlg_gemm_op", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
+              "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
     getattr(_lib, _name).restype = _i32
 
 
@@ -220,6 +232,51 @@ def tlg_gemm_op(A: torch.Tensor, B: torch.Tensor, op_a: str = "N", op_b: str = "
                             pb, ldb, bias.data_ptr() if bias is not None else None, pc, ldc, o, epi,
                             ctypes.byref(cfg) if cfg is not None else None, ws_ptr, ws_bytes,
                             _stream_handle(stream, A, B, C)), "tlg_gemm_op")
+    return C
+
+
+def tlg_gemm_fused(A: torch.Tensor, B: torch.Tensor, op_a: str = "N", op_b: str = "N",
+                   bias: torch.Tensor | None = None, activation: str = "none",
+                   residual: torch.Tensor | None = None, C: torch.Tensor | None = None,
+                   out: str = "f16", config: dict | None = None,
+                   workspace: torch.Tensor | None = None, stream=None):
+    """C = act(op(A).op(B) + bias[col]) + residual[row, col].
+
+    ``activation``: "none", "relu" or "gelu" (exact erf form).  ``residual``:
+    an M x N row-major tensor of C's type (fp16 for out="f16", fp32 for
+    out="f32"); it may be ``C`` itself for an in-place residual connection.
+    Operands and ``op_a`` / ``op_b`` as ``tlg_gemm_op``."""
+    at, bt = op_a.upper() == "T", op_b.upper() == "T"
+    if A.dtype != torch.float16 or B.dtype != torch.float16:
+        raise TypeError("A and B must be fp16")
+    M, K = (A.shape[1], A.shape[0]) if at else tuple(A.shape)
+    K2, N = (B.shape[1], B.shape[0]) if bt else tuple(B.shape)
+    if K != K2:
+        raise ValueError(f"inner dimensions differ: op(A) is {M}x{K}, op(B) is {K2}x{N}")
+    if activation not in _ACT:
+        raise ValueError(f"activation must be one of {sorted(_ACT)}")
+    o = TLG_OUT_F32 if out == "f32" else TLG_OUT_F16
+    cdt = torch.float32 if o == TLG_OUT_F32 else torch.float16
+    C = _out(C, M, N, cdt, A)
+    if bias is not None and (bias.dtype != torch.float16 or bias.dim() != 1 or bias.numel() != N
+                             or (N > 1 and bias.stride(0) != 1)):
+        raise ValueError(f"bias must be a contiguous fp16 vector of length {N}")
+    epi = tlg_fused_epilogue(bias.data_ptr() if bias is not None else None, _ACT[activation], None, 0)
+    if residual is not None:
+        if residual.dtype != cdt or tuple(residual.shape) != (M, N):
+            raise ValueError(f"residual must be {cdt} of shape ({M}, {N})")
+        epi.residual, epi.ldr = _mat(residual, "residual")
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    pc, ldc = _mat(C, "C")
+    cfg = tlg_config(**{k: int(v) for k, v in config.items()}) if config is not None else None
+    ws_ptr, ws_bytes = (None, 0)
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check(_lib.tlg_gemm_fused(M, N, K, TLG_OP_T if at else TLG_OP_N, pa, lda, TLG_OP_T if bt else TLG_OP_N,
+                               pb, ldb, ctypes.byref(epi), pc, ldc, o,
+                               ctypes.byref(cfg) if cfg is not None else None, ws_ptr, ws_bytes,
+                               _stream_handle(stream, A, B, C)), "tlg_gemm_fused")
     return C
 
 

@@ -113,11 +113,15 @@ constexpr KernelCfg kBuilt[] = {{1, 64, 8, 0.35, 0, true},   {1, 128, 6, 0.60, 0
 constexpr int kNumBuilt = sizeof(kBuilt) / sizeof(kBuilt[0]);
 static_assert(kNumBuilt == kNumVariants, "one launcher table entry per built variant");
 
-const VariantFns &fns_for(int idx, bool f16, bool bias_relu, bool at = false, bool bt = false,
+// ek: the epilogue kind (kEpiNone, kEpiFused, kEpiBiasRelu; the last is built
+// for an fp16 C only).
+const VariantFns &fns_for(int idx, bool f16, int ek, bool at = false, bool bt = false,
                           bool plain = false) {
   static const LayoutTables *const layouts[4] = {&kLayoutNN, &kLayoutNT, &kLayoutTN, &kLayoutTT};
   const LayoutTables &t = *layouts[(at ? 2 : 0) + (bt ? 1 : 0)];
-  const int kind = !f16 ? 0 : (bias_relu ? 2 : 1);
+  int kind = f16 ? kKindF16 : kKindF32;
+  if (ek == kEpiFused) kind = f16 ? kKindF16Epi : kKindF32Epi;
+  if (ek == kEpiBiasRelu) kind = f16 ? kKindF16BiasRelu : kKindF32Epi;
   return plain ? t.plain[idx][kind] : t.tma[idx][kind];
 }
 
@@ -181,7 +185,7 @@ struct Resolved {
 // area over its sustained fraction of the MMA peak, per SM).
 // at / bt select the operand-layout instantiation whose launch attributes are
 // prepared (the schedule itself does not depend on the layout).
-tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, bool bias_relu,
+tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, int ek,
                    bool at, bool bt, bool plain, const tlg_config *req, size_t ws_bytes,
                    Resolved *out) {
   const int num_kb = static_cast<int>((K + kBK - 1) / kBK);
@@ -202,7 +206,7 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
     if (plain && !k.plain_loads) continue;
     shape_exists = true;
     int resident = 0;
-    const tlg_status us = fns_for(i, f16, bias_relu, at, bt, plain).units(dev, sms, &resident);
+    const tlg_status us = fns_for(i, f16, ek, at, bt, plain).units(dev, sms, &resident);
     if (us != TLG_OK) return us;
     if (r.max_ctas > 0) resident = std::max(1, std::min(resident, r.max_ctas / k.cta_group));
     const int64_t tile_m = 128 * k.cta_group;
@@ -250,15 +254,58 @@ bool encode_2d(CUtensorMap *tm, CUtensorMapDataType dtype, const void *base, uin
   return r == CUDA_SUCCESS;
 }
 
-template <bool OUT_F16, bool BIAS_RELU>
-tlg_status launch_fill(void *C, int64_t ldc, const void *bias, int M, int N, cudaStream_t s) {
+static_assert(kActNone == TLG_ACT_NONE && kActRelu == TLG_ACT_RELU && kActGelu == TLG_ACT_GELU,
+              "the kernels' activation codes are tlg_activation's values");
+
+// The epilogue of one call, from either interface: bias, activation and
+// residual, and whether the fused-epilogue kernels run at all.
+struct Epi {
+  bool fused = false;
+  const void *bias = nullptr;
+  int act = kActNone;
+  const void *R = nullptr;
+  int64_t ldr = 0;
+};
+
+// tlg_gemm_ex's selector: TLG_EPI_BIAS_RELU is the bias, then the ReLU, fp16 C only.
+tlg_status legacy_epilogue(tlg_out out, tlg_epilogue epi, const void *bias, Epi *e) {
+  if (out != TLG_OUT_F32 && out != TLG_OUT_F16) return TLG_ERR_INVALID_ARG;
+  if (epi != TLG_EPI_NONE && epi != TLG_EPI_BIAS_RELU) return TLG_ERR_INVALID_ARG;
+  if (epi == TLG_EPI_BIAS_RELU && out != TLG_OUT_F16) return TLG_ERR_UNSUPPORTED;
+  if ((epi == TLG_EPI_BIAS_RELU) != (bias != nullptr)) return TLG_ERR_INVALID_ARG;
+  *e = Epi{};
+  if (epi == TLG_EPI_BIAS_RELU) {
+    e->fused = true;
+    e->bias = bias;
+    e->act = kActRelu;
+  }
+  return TLG_OK;
+}
+
+// tlg_gemm_fused's descriptor.  An empty one (or NULL) runs the plain kernels.
+tlg_status fused_epilogue(tlg_out out, const tlg_fused_epilogue *d, Epi *e) {
+  if (out != TLG_OUT_F32 && out != TLG_OUT_F16) return TLG_ERR_INVALID_ARG;
+  *e = Epi{};
+  if (d == nullptr) return TLG_OK;
+  if (d->activation != TLG_ACT_NONE && d->activation != TLG_ACT_RELU &&
+      d->activation != TLG_ACT_GELU)
+    return TLG_ERR_INVALID_ARG;
+  e->bias = d->bias;
+  e->act = d->activation;
+  e->R = d->residual;
+  e->ldr = d->ldr;
+  e->fused = e->bias != nullptr || e->act != kActNone || e->R != nullptr;
+  return TLG_OK;
+}
+
+template <bool OUT_F16, bool EPI>
+tlg_status launch_fill(void *C, int64_t ldc, const Epi &e, int M, int N, cudaStream_t s) {
   const int64_t total = static_cast<int64_t>(M) * N;
   const int threads = 256;
   const int blocks = static_cast<int>(total / threads + 1 > 4096 ? 4096 : total / threads + 1);
-  fill_empty_k_kernel<OUT_F16, BIAS_RELU><<<blocks, threads, 0, s>>>(
-      C, ldc, static_cast<const __half *>(bias), M, N);
-  const cudaError_t e = cudaPeekAtLastError();
-  if (e != cudaSuccess) {
+  fill_empty_k_kernel<OUT_F16, EPI><<<blocks, threads, 0, s>>>(
+      C, ldc, static_cast<const __half *>(e.bias), e.act, e.R, e.ldr, M, N);
+  if (cudaPeekAtLastError() != cudaSuccess) {
     cudaGetLastError();
     return TLG_ERR_CUDA;
   }
@@ -269,12 +316,10 @@ tlg_status launch_fill(void *C, int64_t ldc, const void *bias, int M, int N, cud
 // at / bt: A stored K x M (lda >= M), B stored N x K (ldb >= K), the product
 // using their transposes.
 tlg_status check_args(int64_t M, int64_t N, int64_t K, bool at, const void *A, int64_t lda,
-                      bool bt, const void *B, int64_t ldb, const void *bias, const void *C,
-                      int64_t ldc, tlg_out out, tlg_epilogue epi) {
+                      bool bt, const void *B, int64_t ldb, const Epi &e, const void *C,
+                      int64_t ldc, tlg_out out) {
   if (out != TLG_OUT_F32 && out != TLG_OUT_F16) return TLG_ERR_INVALID_ARG;
-  if (epi != TLG_EPI_NONE && epi != TLG_EPI_BIAS_RELU) return TLG_ERR_INVALID_ARG;
-  if (epi == TLG_EPI_BIAS_RELU && out != TLG_OUT_F16) return TLG_ERR_UNSUPPORTED;
-  if ((epi == TLG_EPI_BIAS_RELU) != (bias != nullptr)) return TLG_ERR_INVALID_ARG;
+  const void *bias = e.bias;
   if (M < 0 || N < 0 || K < 0) return TLG_ERR_INVALID_ARG;
   // TMA coordinates and tile indices are 32-bit: keep every extent (plus one tile) below 2^31.
   const int64_t kMax = 0x7fffffff - 256;
@@ -311,15 +356,28 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, bool at, const void *A, i
     const uintptr_t s0 = reinterpret_cast<uintptr_t>(bias);
     if (overlaps(c0, c1, s0, s0 + static_cast<uintptr_t>(2 * N))) return TLG_ERR_INVALID_ARG;
   }
+  if (e.R != nullptr) {
+    // The residual has C's type.  It may be C itself (same base and row
+    // stride: each element is read before the one thread that owns it writes
+    // it); any other overlap with C would race.
+    if (misaligned(e.R, static_cast<uintptr_t>(osz))) return TLG_ERR_ALIGNMENT;
+    if (e.ldr < N) return TLG_ERR_INVALID_ARG;
+    if (e.ldr > (int64_t(1) << 36)) return TLG_ERR_UNSUPPORTED;
+    if (!(e.R == C && e.ldr == ldc)) {
+      uintptr_t r0, r1;
+      extent(e.R, M, N, e.ldr, osz, &r0, &r1);
+      if (overlaps(c0, c1, r0, r1)) return TLG_ERR_INVALID_ARG;
+    }
+  }
   return TLG_OK;
 }
 
 // ws/ws_bytes: scratch for the split-K tail (nullptr/0: none).
 tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, int64_t lda,
-                     bool bt, const void *B, int64_t ldb, const void *bias, void *C, int64_t ldc,
-                     tlg_out out, tlg_epilogue epi, const tlg_config *req, void *ws,
-                     size_t ws_bytes, void *stream) {
-  const tlg_status hs = check_args(M, N, K, at, A, lda, bt, B, ldb, bias, C, ldc, out, epi);
+                     bool bt, const void *B, int64_t ldb, const Epi &e, void *C, int64_t ldc,
+                     tlg_out out, const tlg_config *req, void *ws, size_t ws_bytes, void *stream) {
+  const tlg_status hs = check_args(M, N, K, at, A, lda, bt, B, ldb, e, C, ldc, out);
+  const void *bias = e.bias;
   if (hs != TLG_OK || M == 0 || N == 0) return hs;
   const int64_t osz = out == TLG_OUT_F32 ? 4 : 2;
   if (ws == nullptr) ws_bytes = 0;
@@ -336,6 +394,11 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
       if (overlaps(w0, w0 + ws_bytes, a0, a1) || overlaps(w0, w0 + ws_bytes, b0, b1))
         return TLG_ERR_INVALID_ARG;
     }
+    if (e.R != nullptr) {
+      uintptr_t r0, r1;
+      extent(e.R, M, N, e.ldr, osz, &r0, &r1);
+      if (overlaps(w0, w0 + ws_bytes, r0, r1)) return TLG_ERR_INVALID_ARG;
+    }
   }
 
   // ---- device checks
@@ -347,23 +410,31 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   if (K > 0 && (!device_accessible(A, dev) || !device_accessible(B, dev)))
     return TLG_ERR_INVALID_ARG;
   if (bias != nullptr && !device_accessible(bias, dev)) return TLG_ERR_INVALID_ARG;
+  if (e.R != nullptr && !device_accessible(e.R, dev)) return TLG_ERR_INVALID_ARG;
   if (ws != nullptr && !device_accessible(ws, dev)) return TLG_ERR_INVALID_ARG;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool f16 = out == TLG_OUT_F16;
-  const bool br = epi == TLG_EPI_BIAS_RELU;
+  const bool fused = e.fused;
   if (K == 0) {
-    if (!f16) return launch_fill<false, false>(C, ldc, bias, int(M), int(N), s);
-    if (br) return launch_fill<true, true>(C, ldc, bias, int(M), int(N), s);
-    return launch_fill<true, false>(C, ldc, bias, int(M), int(N), s);
+    if (f16)
+      return fused ? launch_fill<true, true>(C, ldc, e, int(M), int(N), s)
+                   : launch_fill<true, false>(C, ldc, e, int(M), int(N), s);
+    return fused ? launch_fill<false, true>(C, ldc, e, int(M), int(N), s)
+                 : launch_fill<false, false>(C, ldc, e, int(M), int(N), s);
   }
+  // Bias + ReLU alone (an fp16 C, no residual) runs the kernels built for it.
+  const int ek = !fused ? kEpiNone
+                        : (f16 && e.bias != nullptr && e.act == kActRelu && e.R == nullptr)
+                              ? kEpiBiasRelu
+                              : kEpiFused;
 
   // TMA needs 16-byte aligned bases and row strides.
   const bool plain = !(aligned16(A) && aligned16(B) && (lda * 2) % 16 == 0 && (ldb * 2) % 16 == 0);
   const bool c_plain = !(aligned16(C) && (ldc * osz) % 16 == 0);
   Resolved rv;
   const tlg_status rs =
-      resolve(dev, info.sm_count, M, N, K, f16, br, at, bt, plain, req, ws_bytes, &rv);
+      resolve(dev, info.sm_count, M, N, K, f16, ek, at, bt, plain, req, ws_bytes, &rv);
   if (rs != TLG_OK) return rs;
   if (rv.sched.workspace > ws_bytes) return TLG_ERR_INVALID_ARG;  // a forced split needs scratch
 
@@ -410,7 +481,11 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   p.ldb = ldb;
   p.c_plain = c_plain ? 1 : 0;
   p.bias_aligned = (bias != nullptr && aligned16(bias)) ? 1 : 0;
-  return fns_for(rv.idx, f16, br, at, bt, plain)
+  p.act = e.act;
+  p.R = e.R;
+  p.ldr = e.ldr;
+  p.r_vec = (e.R != nullptr && aligned16(e.R) && (e.ldr * osz) % 16 == 0) ? 1 : 0;
+  return fns_for(rv.idx, f16, ek, at, bt, plain)
       .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
 }
 
@@ -464,7 +539,10 @@ tlg_status resolve_public(int64_t M, int64_t N, int64_t K, tlg_out out, tlg_epil
   const tlg_status ds = current_device(&dev, &info);
   if (ds != TLG_OK) return ds;
   return resolve(dev, info.sm_count, std::max<int64_t>(M, 1), std::max<int64_t>(N, 1),
-                 std::max<int64_t>(K, 1), out == TLG_OUT_F16, epilogue == TLG_EPI_BIAS_RELU, false,
+                 std::max<int64_t>(K, 1), out == TLG_OUT_F16,
+                 epilogue != TLG_EPI_BIAS_RELU ? kEpiNone
+                                               : (out == TLG_OUT_F16 ? kEpiBiasRelu : kEpiFused),
+                 false,
                  false, false, req, ws_bytes, rv);
 }
 
@@ -494,50 +572,76 @@ extern "C" {
 
 tlg_status tlg_gemm_f16f32(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                            const void *B, int64_t ldb, float *C, int64_t ldc, void *stream) {
-  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, nullptr, C, ldc, TLG_OUT_F32,
-                   TLG_EPI_NONE, nullptr, nullptr, 0, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, Epi{}, C, ldc, TLG_OUT_F32, nullptr,
+                   nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_f16f16(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                            const void *B, int64_t ldb, void *C, int64_t ldc, void *stream) {
-  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, nullptr, C, ldc, TLG_OUT_F16,
-                   TLG_EPI_NONE, nullptr, nullptr, 0, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, Epi{}, C, ldc, TLG_OUT_F16, nullptr,
+                   nullptr, 0, stream);
 }
 
 tlg_status tlg_gemm_bias_relu_f16(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                                   const void *B, int64_t ldb, const void *bias, void *C,
                                   int64_t ldc, void *stream) {
   if (bias == nullptr && M > 0 && N > 0) return TLG_ERR_INVALID_ARG;
-  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, TLG_OUT_F16,
-                   TLG_EPI_BIAS_RELU, nullptr, nullptr, 0, stream);
+  Epi e;
+  const tlg_status es = legacy_epilogue(TLG_OUT_F16, TLG_EPI_BIAS_RELU, bias, &e);
+  if (es != TLG_OK) return es;
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, e, C, ldc, TLG_OUT_F16, nullptr, nullptr,
+                   0, stream);
 }
 
 tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
                        int64_t ldb, const void *bias, void *C, int64_t ldc, tlg_out out,
                        tlg_epilogue epilogue, const tlg_config *config, void *workspace,
                        size_t workspace_bytes, void *stream) {
-  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, out, epilogue, config,
-                   workspace, workspace_bytes, stream);
+  Epi e;
+  const tlg_status es = legacy_epilogue(out, epilogue, bias, &e);
+  if (es != TLG_OK) return es;
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, e, C, ldc, out, config, workspace,
+                   workspace_bytes, stream);
 }
 
 tlg_status tlg_gemm_op(int64_t M, int64_t N, int64_t K, tlg_op op_a, const void *A, int64_t lda,
                        tlg_op op_b, const void *B, int64_t ldb, const void *bias, void *C,
                        int64_t ldc, tlg_out out, tlg_epilogue epilogue, const tlg_config *config,
                        void *workspace, size_t workspace_bytes, void *stream) {
+  Epi e;
+  const tlg_status es = legacy_epilogue(out, epilogue, bias, &e);
+  if (es != TLG_OK) return es;
   if ((op_a != TLG_OP_N && op_a != TLG_OP_T) || (op_b != TLG_OP_N && op_b != TLG_OP_T))
     return TLG_ERR_INVALID_ARG;
-  return gemm_impl(M, N, K, op_a == TLG_OP_T, A, lda, op_b == TLG_OP_T, B, ldb, bias, C, ldc, out,
-                   epilogue, config, workspace, workspace_bytes, stream);
+  return gemm_impl(M, N, K, op_a == TLG_OP_T, A, lda, op_b == TLG_OP_T, B, ldb, e, C, ldc, out,
+                   config, workspace, workspace_bytes, stream);
+}
+
+tlg_status tlg_gemm_fused(int64_t M, int64_t N, int64_t K, tlg_op op_a, const void *A,
+                          int64_t lda, tlg_op op_b, const void *B, int64_t ldb,
+                          const tlg_fused_epilogue *epilogue, void *C, int64_t ldc, tlg_out out,
+                          const tlg_config *config, void *workspace, size_t workspace_bytes,
+                          void *stream) {
+  Epi e;
+  const tlg_status es = fused_epilogue(out, epilogue, &e);
+  if (es != TLG_OK) return es;
+  if ((op_a != TLG_OP_N && op_a != TLG_OP_T) || (op_b != TLG_OP_N && op_b != TLG_OP_T))
+    return TLG_ERR_INVALID_ARG;
+  return gemm_impl(M, N, K, op_a == TLG_OP_T, A, lda, op_b == TLG_OP_T, B, ldb, e, C, ldc, out,
+                   config, workspace, workspace_bytes, stream);
 }
 
 tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K, const void *A, int64_t lda,
                                const void *B, int64_t ldb, const void *bias, void *C, int64_t ldc,
                                tlg_out out, tlg_epilogue epilogue, const tlg_config *config,
                                void *stream) {
+  Epi e;
+  const tlg_status es = legacy_epilogue(out, epilogue, bias, &e);
+  if (es != TLG_OK) return es;
   const bool split = config != nullptr && config->split_k >= 2;
   if (!split)  // no scratch needed: exactly tlg_gemm_ex without a workspace
-    return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, out, epilogue, config,
-                     nullptr, 0, stream);
+    return gemm_impl(M, N, K, false, A, lda, false, B, ldb, e, C, ldc, out, config, nullptr, 0,
+                     stream);
   // Reject a schedule whose scratch would not fit before touching anything.
   if (M > 0 && N > 0 && K > 0) {
     Resolved rv;
@@ -554,8 +658,8 @@ tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K, const void *A, i
     cudaGetLastError();
     return TLG_ERR_CUDA;
   }
-  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, bias, C, ldc, out, epilogue, config,
-                   scratch, kStaticScratchBytes, stream);
+  return gemm_impl(M, N, K, false, A, lda, false, B, ldb, e, C, ldc, out, config, scratch,
+                   kStaticScratchBytes, stream);
 }
 
 tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,

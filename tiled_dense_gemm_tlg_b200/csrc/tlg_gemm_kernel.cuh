@@ -93,6 +93,11 @@ struct GemmParams {
   int64_t lda, ldb;
   int c_plain;       // C cannot be written by TMA (base or row stride not 16-byte aligned)
   int bias_aligned;  // the bias may be read 16 bytes at a time
+  // Fused epilogue (kernels built with kEpiFused): C = act(acc + bias[col]) + R[row, col].
+  int act;           // kActNone, kActRelu or kActGelu
+  const void *R;     // residual in C's type, or nullptr; may be C itself (same ldc)
+  int64_t ldr;
+  int r_vec;         // R's base and row stride are 16-byte aligned
 };
 
 // One unit of work: a tile, or one k-slice of a tail tile.
@@ -148,30 +153,239 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int gro
   nb = r / gm;
 }
 
-// Adds bias[col0 + j] (j < 32) to v and applies the ReLU.  Bias entries at
-// columns >= N are not read (those outputs are clipped by the store).
-__device__ __forceinline__ void bias_relu_32(const __half *__restrict__ bias, int col0, int N,
-                                             bool aligned, float (&v)[32]) {
-  if (aligned && col0 + 32 <= N) {
-    const uint4 *bp = reinterpret_cast<const uint4 *>(bias + col0);
+// Epilogue kinds a kernel is built with: the plain product; the general fused
+// epilogue (bias, activation and residual chosen at run time); and bias +
+// ReLU alone, whose code is a small part of the general one.  The epilogue
+// warps share each SM sub-partition's instruction cache with the producer and
+// MMA warps, and the general epilogue's larger code measurably slows the main
+// loop even where it does the same work, so the common bias + ReLU case gets
+// its own build.
+constexpr int kEpiNone = 0;
+constexpr int kEpiFused = 1;
+constexpr int kEpiBiasRelu = 2;
+
+// Activation codes of the fused epilogue (the values of tlg_activation).
+constexpr int kActNone = 0;
+constexpr int kActRelu = 1;
+constexpr int kActGelu = 2;
+
+// Hardware approximations (PTX rcp.approx / ex2.approx, flushing subnormals).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// GELU in its exact form x * Phi(x), Phi the standard normal CDF, in fp32.
+// Phi(-|x|) = erfc(z) / 2 with z = |x| / sqrt 2, and erfc is taken from
+// Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
+// (Hastings' rational approximation, |error| <= 1.5e-7 for z >= 0):
+//   erfc(z) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),
+//   t = 1 / (1 + p z).
+// Here 1/sqrt 2 is folded into p, the 1/2 into the a_i, and exp(-z^2) =
+// 2^(x^2 * (-log2(e) / 2)).  That gives Phi(-|x|) directly (no cancellation
+// in the negative tail) and Phi(|x|) = 1 - Phi(-|x|).  Branch-free, so the 32
+// values a thread holds are evaluated side by side; every instruction counts,
+// since the epilogue's arithmetic competes with the tensor pipe for the SM.
+__device__ __forceinline__ float gelu_erf(float x) {
+  constexpr float kPz = 0.3275911f * 0.70710678118654752f;
+  constexpr float kH1 = 0.5f * 0.254829592f, kH2 = 0.5f * -0.284496736f,
+                  kH3 = 0.5f * 1.421413741f, kH4 = 0.5f * -1.453152027f,
+                  kH5 = 0.5f * 1.061405429f;
+  constexpr float kE = -0.5f * 1.4426950408889634f;
+  const float t = rcp_approx(fmaf(kPz, fabsf(x), 1.0f));
+  const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kH5, kH4), kH3), kH2), kH1);
+  const float q = poly * ex2_approx(x * x * kE);  // Phi(-|x|)
+  return x * (x < 0.0f ? q : 1.0f - q);
+}
+
+__device__ __forceinline__ float activate(int act, float x) {
+  if (act == kActRelu) return fmaxf(x, 0.0f);
+  if (act == kActGelu) return gelu_erf(x);
+  return x;
+}
+
+// The activation over 32 values; `act` is the same for every thread, so the
+// branch does not diverge.
+__device__ __forceinline__ void activate_32(int act, float (&v)[32]) {
+  if (act == kActRelu) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 w = __ldg(bp + q);
-      const __half2 *h = reinterpret_cast<const __half2 *>(&w);
+    for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
+  } else if (act == kActGelu) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h[e]);
-        v[q * 8 + 2 * e] += f.x;
-        v[q * 8 + 2 * e + 1] += f.y;
+    for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+  }
+}
+
+// Adds the residual R[row, col0 + j] (j < 32), read in C's type.  Rows >= M
+// and columns >= N are not read.  R may be C itself: every element is read
+// here, by the one thread that later writes it, before that write, and no
+// other thread touches it.  The loads are ordinary (not the read-only path)
+// for that reason.
+template <bool OUT_F16>
+__device__ __forceinline__ void add_residual_32(const GemmParams &p, int row, int col0,
+                                                float (&v)[32]) {
+  if (row >= p.M) return;
+  if constexpr (OUT_F16) {
+    const __half *r = static_cast<const __half *>(p.R) + static_cast<int64_t>(row) * p.ldr + col0;
+    if (p.r_vec && col0 + 32 <= p.N) {
+      const uint4 *q = reinterpret_cast<const uint4 *>(r);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 w = q[c];
+        const __half2 *h = reinterpret_cast<const __half2 *>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(h[e]);
+          v[c * 8 + 2 * e] += f.x;
+          v[c * 8 + 2 * e + 1] += f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < p.N) v[j] += __half2float(r[j]);
+    }
+  } else {
+    const float *r = static_cast<const float *>(p.R) + static_cast<int64_t>(row) * p.ldr + col0;
+    if (p.r_vec && col0 + 32 <= p.N) {
+      const float4 *q = reinterpret_cast<const float4 *>(r);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 w = q[c];
+        v[4 * c] += w.x;
+        v[4 * c + 1] += w.y;
+        v[4 * c + 2] += w.z;
+        v[4 * c + 3] += w.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < p.N) v[j] += r[j];
+    }
+  }
+}
+
+// Epilogue input of one 64-column piece of this lane's row loaded ahead of
+// its use: the fp16 residual row piece (128 bytes, 16 at a time), whose DRAM
+// latency would otherwise stall every piece.  The bias (a few KB, reused by
+// every row) and an fp32 residual are read in epi_apply: holding them too
+// would push the epilogue past the register file.  Pieces the vector loads
+// cannot serve (ragged or unaligned) are also read in epi_apply.  ON = false
+// (an fp32 C, or the plain-load kernels, whose extra loader warps leave each
+// thread fewer registers) keeps nothing and reads the residual at its use.
+template <bool ON>
+struct EpiIn {
+  uint4 r[ON ? 8 : 1];  // R[row, col0 .. col0+63], fp16
+  bool has_r;
+};
+
+template <bool ON>
+__device__ __forceinline__ void epi_prefetch(const GemmParams &p, int row, int col0,
+                                             EpiIn<ON> &in) {
+  in.has_r = ON && p.R != nullptr && p.r_vec != 0 && col0 + 64 <= p.N && row < p.M;
+  if constexpr (ON) {
+    if (in.has_r) {
+      // Ordinary loads, not the read-only path: R may be C itself.
+      const uint4 *q = reinterpret_cast<const uint4 *>(static_cast<const __half *>(p.R) +
+                                                       static_cast<int64_t>(row) * p.ldr + col0);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) in.r[c] = q[c];
+    }
+  }
+}
+
+// The bias of one tile's columns, spread over the warp: lane l holds columns
+// [l * CPL, (l + 1) * CPL) of the tile (CPL = tile width / 32) as packed fp16
+// pairs.  Loaded once per tile, before the accumulator is ready, so no piece
+// of the epilogue waits on a bias load; a piece gets its columns with warp
+// shuffles.
+template <int CPL>
+struct BiasSlice {
+  static_assert(CPL >= 2 && CPL % 2 == 0, "whole fp16 pairs per lane");
+  uint32_t w[CPL / 2];
+};
+
+template <int CPL>
+__device__ __forceinline__ void load_bias_slice(const GemmParams &p, int tile_col0, int lane,
+                                                BiasSlice<CPL> &s) {
+  const int c = tile_col0 + lane * CPL;
+  if (p.bias_aligned != 0 && c + CPL <= p.N) {
+    // c * 2 bytes is a multiple of CPL * 2 >= 4 and the bias base is 16-byte aligned.
+    if constexpr (CPL == 2) {
+      s.w[0] = __ldg(reinterpret_cast<const unsigned int *>(p.bias + c));
+    } else if constexpr (CPL == 4) {
+      const uint2 x = __ldg(reinterpret_cast<const uint2 *>(p.bias + c));
+      s.w[0] = x.x;
+      s.w[1] = x.y;
+    } else {
+#pragma unroll
+      for (int q = 0; q < CPL / 8; ++q) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(p.bias + c) + q);
+        s.w[4 * q] = x.x;
+        s.w[4 * q + 1] = x.y;
+        s.w[4 * q + 2] = x.z;
+        s.w[4 * q + 3] = x.w;
       }
     }
   } else {
+    const unsigned short *b = reinterpret_cast<const unsigned short *>(p.bias);
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (col0 + j < N) v[j] += __half2float(bias[col0 + j]);
+    for (int i = 0; i < CPL / 2; ++i) {
+      const uint32_t lo = c + 2 * i < p.N ? b[c + 2 * i] : 0u;
+      const uint32_t hi = c + 2 * i + 1 < p.N ? b[c + 2 * i + 1] : 0u;
+      s.w[i] = lo | (hi << 16);
+    }
   }
+}
+
+// v[j] += bias[tile column t0 + j], j < 32, t0 a multiple of 32, from the slice.
+template <int CPL>
+__device__ __forceinline__ void add_bias_slice_32(const BiasSlice<CPL> &s, int t0,
+                                                  float (&v)[32]) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
+  for (int jj = 0; jj < 16; ++jj) {
+    // columns t0 + 2jj and t0 + 2jj + 1 sit in one word of lane (t0 + 2jj) / CPL
+    const uint32_t w = __shfl_sync(0xffffffffu, s.w[((2 * jj) % CPL) / 2], (t0 + 2 * jj) / CPL);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+    v[2 * jj] += f.x;
+    v[2 * jj + 1] += f.y;
+  }
+}
+
+// The fused epilogue on half `half` (columns col0 + 32*half ..) of a
+// 64-column piece at tile column tcol: + bias, activation, + residual.  Done
+// one half at a time so that the first half is packed for the store (and its
+// registers freed) before the second half's activation runs.
+template <bool OUT_F16, bool ON, int CPL>
+__device__ __forceinline__ void epi_apply_32(const GemmParams &p, const EpiIn<ON> &in,
+                                             const BiasSlice<CPL> &bias, int row, int col0,
+                                             int tcol, int half, float (&v)[32]) {
+  const int c0 = col0 + 32 * half;
+  if (p.bias != nullptr) add_bias_slice_32<CPL>(bias, tcol + 32 * half, v);
+  activate_32(p.act, v);
+  if (p.R != nullptr) {
+    if (ON && in.has_r) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const __half2 *h = reinterpret_cast<const __half2 *>(&in.r[4 * half + c]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(h[e]);
+          v[c * 8 + 2 * e] += f.x;
+          v[c * 8 + 2 * e + 1] += f.y;
+        }
+      }
+    } else {
+      add_residual_32<OUT_F16>(p, row, c0, v);
+    }
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -281,7 +495,7 @@ __device__ __forceinline__ uint32_t mnmajor_offset(int mn, int k) {
 // LSU: the operands are loaded by kLoaderWarps extra warps with 2-byte global
 // loads into the same swizzled shared-memory layouts, for strides and bases
 // the TMA unit cannot describe; the tensor-core pipeline is unchanged.
-template <int CG, int BN, int STAGES, bool OUT_F16, bool BIAS_RELU, int NH = 1, bool AT = false,
+template <int CG, int BN, int STAGES, bool OUT_F16, int EK, int NH = 1, bool AT = false,
           bool BT = false, bool LSU = false>
 __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -619,19 +833,36 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     uint32_t acc_phase = 0;
     uint32_t boxes_used = 0;
 
-    // Bias, ReLU, output rounding and the store of one 32-row x 64-column
-    // piece (this lane's row, columns col0 .. col0+63).
-    auto emit64 = [&](float (&va)[32], float (&vb)[32], int box_row0, int col0) {
-      if constexpr (BIAS_RELU) {
-        bias_relu_32(p.bias, col0, p.N, p.bias_aligned != 0, va);
-        bias_relu_32(p.bias, col0 + 32, p.N, p.bias_aligned != 0, vb);
+    // Fused epilogue (bias, activation, residual: inputs prefetched in `in`),
+    // output rounding and the store of one 32-row x 64-column piece (this
+    // lane's row, columns col0 .. col0+63).  next_col0 >= 0: once `in` is
+    // used, load the epilogue inputs of the piece at next_col0 into it, so
+    // their latency passes while this piece is stored.
+    constexpr int kCPL = kTileN / 32;  // bias columns per lane
+    constexpr bool kPrefR = EK == kEpiFused && OUT_F16 && !LSU;  // residual pieces loaded ahead
+    // The epilogue of one 32-column half of a piece (tile columns tcol + 32*half ..).
+    auto epi32 = [&](const EpiIn<kPrefR> &in, const BiasSlice<kCPL> &bias, int row, int col0,
+                     int tcol, int half, float(&v)[32]) {
+      if constexpr (EK == kEpiFused) {
+        epi_apply_32<OUT_F16, kPrefR, kCPL>(p, in, bias, row, col0, tcol, half, v);
+      } else if constexpr (EK == kEpiBiasRelu) {
+        add_bias_slice_32<kCPL>(bias, tcol + 32 * half, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
       }
+    };
+    auto emit64 = [&](float (&va)[32], float (&vb)[32], int box_row0, int col0, int tcol,
+                      const BiasSlice<kCPL> &bias, EpiIn<kPrefR> &in, int next_col0) {
       if constexpr (OUT_F16) {
         uint32_t h[32];  // 64 fp16 values, round to nearest even
+        epi32(in, bias, box_row0 + lane, col0, tcol, 0, va);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          h[j] = pack_half2(va[2 * j], va[2 * j + 1]);
-          h[16 + j] = pack_half2(vb[2 * j], vb[2 * j + 1]);
+        for (int j = 0; j < 16; ++j) h[j] = pack_half2(va[2 * j], va[2 * j + 1]);
+        epi32(in, bias, box_row0 + lane, col0, tcol, 1, vb);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) h[16 + j] = pack_half2(vb[2 * j], vb[2 * j + 1]);
+        if constexpr (kPrefR) {
+          if (next_col0 >= 0) epi_prefetch<kPrefR>(p, box_row0 + lane, next_col0, in);
         }
         if (p.c_plain || (!p.n_aligned && col0 + kBoxCols > p.N)) {
           store_row_tail<true>(p, box_row0 + lane, col0, h);
@@ -649,6 +880,11 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         }
         ++boxes_used;
       } else {
+        epi32(in, bias, box_row0 + lane, col0, tcol, 0, va);
+        epi32(in, bias, box_row0 + lane, col0, tcol, 1, vb);
+        if constexpr (kPrefR) {
+          if (next_col0 >= 0) epi_prefetch<kPrefR>(p, box_row0 + lane, next_col0, in);
+        }
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (col0 + half * kBoxCols >= p.N) break;
@@ -676,93 +912,115 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
 
     for (int k = 0; k < n_work; ++k) {
       const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+      const int box_row0 = w.mb * kTileM + box_row0_in_tile;
+      // The tile's bias and the first piece's residual load while the main
+      // loop still runs.
+      EpiIn<kPrefR> in;
+      BiasSlice<kCPL> bias;
+      if constexpr (EK != kEpiNone) {
+        if (p.bias != nullptr && w.nb * kTileN < p.N) load_bias_slice<kCPL>(p, w.nb * kTileN, lane, bias);
+      }
+      if constexpr (kPrefR) {
+        if (w.tail < 0 && box_row0 < p.M && w.nb * kTileN < p.N)
+          epi_prefetch<kPrefR>(p, box_row0 + lane, w.nb * kTileN, in);
+      }
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.limit_ns, kRoleEpilogue,
                      &g_device_error))
         break;
       tc_fence_after_sync();
-      const int box_row0 = w.mb * kTileM + box_row0_in_tile;
       // A k-slice of a tail tile writes its fp32 partial (this warp's 32 rows x
       // kTileN columns, column by column so each store is 128 contiguous bytes).
       float *part = nullptr;
       if (w.tail >= 0)
         part = p.ws + static_cast<int64_t>(((w.tail * p.split + w.slice) * CG + static_cast<int>(rank)) * 4 +
                                            quarter) * (32 * kTileN);
+      // Pass 0 drains the accumulator: it stores the tile, or writes a tail
+      // slice's partial.  Pass 1 runs only in the warp that completes a tail
+      // tile's count: it sums every slice's partial in slice order (a fixed
+      // order: the result does not depend on which slice finished last) and
+      // stores the tile piece.  Both passes share one copy of the epilogue.
+      uint32_t *counter = nullptr;
+      const float *part0 = nullptr;
+      const int64_t slice_stride = static_cast<int64_t>(CG) * 4 * 32 * kTileN;
 #pragma unroll 1
-      for (int tc = 0; tc < kTileN; tc += 64) {
-        const int slot = NH == 1 ? acc : tc / BN;  // TMEM half holding these columns
-        const int ch = tc % BN;
-        uint32_t ra[32], rb[32];
-        __syncwarp();
-        tmem_load_2x32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                               static_cast<uint32_t>(slot * BN + ch),
-                           ra, rb);
-        if (ch + 64 >= BN) {
-          // Last read of this accumulator half: hand it back to the MMA warp
-          // now, before the stores, so the next tile's main loop can start.
-          tc_fence_before_sync();
+      for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1) {
+          if (part == nullptr) break;
+          counter = p.counters + (w.tail * CG + static_cast<int>(rank)) * 4 + quarter;
           __syncwarp();
+          uint32_t before = 0;
           if (lane == 0) {
-            if constexpr (CG == 2)
-              mbar_arrive_cluster(release_bar0 + 8u * slot);
-            else
-              mbar_arrive(release_bar0 + 8u * slot);
+            __threadfence();
+            before = atomicAdd(counter, 1u);
+          }
+          before = __shfl_sync(0xffffffffu, before, 0);
+          if (before != static_cast<uint32_t>(p.split - 1)) break;
+          __threadfence();
+          part0 = p.ws + static_cast<int64_t>(((w.tail * p.split) * CG + static_cast<int>(rank)) * 4 +
+                                              quarter) * (32 * kTileN);
+          if constexpr (kPrefR) {
+            if (box_row0 < p.M && w.nb * kTileN < p.N)
+              epi_prefetch<kPrefR>(p, box_row0 + lane, w.nb * kTileN, in);
           }
         }
-        if (part != nullptr) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            st_global_cg(part + (tc + j) * 32 + lane, __uint_as_float(ra[j]));
-            st_global_cg(part + (tc + 32 + j) * 32 + lane, __uint_as_float(rb[j]));
-          }
-          continue;
-        }
-        const int col0 = w.nb * kTileN + tc;
-        if (box_row0 >= p.M || col0 >= p.N) continue;  // the whole 32 x 64 piece is clipped
-        float va[32], vb[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          va[j] = __uint_as_float(ra[j]);
-          vb[j] = __uint_as_float(rb[j]);
-        }
-        emit64(va, vb, box_row0, col0);
-      }
-      if (part != nullptr) {
-        // Count this slice in; the warp that completes the count sums every
-        // slice's partial in slice order (a fixed order: the result does not
-        // depend on which slice finished last) and stores the tile piece.
-        uint32_t *counter = p.counters + (w.tail * CG + static_cast<int>(rank)) * 4 + quarter;
-        __syncwarp();
-        uint32_t before = 0;
-        if (lane == 0) {
-          __threadfence();
-          before = atomicAdd(counter, 1u);
-        }
-        before = __shfl_sync(0xffffffffu, before, 0);
-        if (before == static_cast<uint32_t>(p.split - 1)) {
-          __threadfence();
-          const float *part0 = p.ws + static_cast<int64_t>(((w.tail * p.split) * CG + static_cast<int>(rank)) * 4 +
-                                                           quarter) * (32 * kTileN);
-          const int64_t slice_stride = static_cast<int64_t>(CG) * 4 * 32 * kTileN;
 #pragma unroll 1
-          for (int ch = 0; ch < kTileN; ch += 64) {
-            const int col0 = w.nb * kTileN + ch;
-            if (box_row0 >= p.M || col0 >= p.N) continue;
-            float va[32], vb[32];
+        for (int tc = 0; tc < kTileN; tc += 64) {
+          const int col0 = w.nb * kTileN + tc;
+          float va[32], vb[32];
+          if (pass == 0) {
+            const int slot = NH == 1 ? acc : tc / BN;  // TMEM half holding these columns
+            const int ch = tc % BN;
+            uint32_t ra[32], rb[32];
+            __syncwarp();
+            tmem_load_2x32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(slot * BN + ch),
+                               ra, rb);
+            if (ch + 64 >= BN) {
+              // Last read of this accumulator half: hand it back to the MMA warp
+              // now, before the stores, so the next tile's main loop can start.
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) {
+                if constexpr (CG == 2)
+                  mbar_arrive_cluster(release_bar0 + 8u * slot);
+                else
+                  mbar_arrive(release_bar0 + 8u * slot);
+              }
+            }
+            if (part != nullptr) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                st_global_cg(part + (tc + j) * 32 + lane, __uint_as_float(ra[j]));
+                st_global_cg(part + (tc + 32 + j) * 32 + lane, __uint_as_float(rb[j]));
+              }
+              continue;
+            }
+            if (box_row0 >= p.M || col0 >= p.N) continue;  // the whole 32 x 64 piece is clipped
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              va[j] = ld_global_cg(part0 + (ch + j) * 32 + lane);
-              vb[j] = ld_global_cg(part0 + (ch + 32 + j) * 32 + lane);
+              va[j] = __uint_as_float(ra[j]);
+              vb[j] = __uint_as_float(rb[j]);
+            }
+          } else {
+            if (box_row0 >= p.M || col0 >= p.N) continue;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              va[j] = ld_global_cg(part0 + (tc + j) * 32 + lane);
+              vb[j] = ld_global_cg(part0 + (tc + 32 + j) * 32 + lane);
             }
             for (int sl = 1; sl < p.split; ++sl) {
               const float *ps = part0 + sl * slice_stride;
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
-                va[j] += ld_global_cg(ps + (ch + j) * 32 + lane);
-                vb[j] += ld_global_cg(ps + (ch + 32 + j) * 32 + lane);
+                va[j] += ld_global_cg(ps + (tc + j) * 32 + lane);
+                vb[j] += ld_global_cg(ps + (tc + 32 + j) * 32 + lane);
               }
             }
-            emit64(va, vb, box_row0, col0);
           }
+          const int next_col0 = (tc + 64 < kTileN && col0 + 64 < p.N) ? col0 + 64 : -1;
+          emit64(va, vb, box_row0, col0, tc, bias, in, next_col0);
+        }
+        if (pass == 1) {
           __syncwarp();
           if (lane == 0) atomicExch(counter, 0u);  // ready for the next call
         }
@@ -791,15 +1049,23 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
   }
 }
 
-// C = 0 (or fp16(max(bias[col], 0))) for K == 0, where the sum over k is empty.
-template <bool OUT_F16, bool BIAS_RELU>
-__global__ void fill_empty_k_kernel(void *C, int64_t ldc, const __half *bias, int M, int N) {
+// K == 0, where the sum over k is empty: C = 0, or with the fused epilogue
+// C = act(bias[col]) + R[row, col] (each element read and written by one thread).
+template <bool OUT_F16, bool EPI>
+__global__ void fill_empty_k_kernel(void *C, int64_t ldc, const __half *bias, int act,
+                                    const void *R, int64_t ldr, int M, int N) {
   const int64_t total = static_cast<int64_t>(M) * N;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = i / N, c = i % N;
     float v = 0.0f;
-    if constexpr (BIAS_RELU) v = fmaxf(__half2float(bias[c]), 0.0f);
+    if constexpr (EPI) {
+      if (bias != nullptr) v = __half2float(bias[c]);
+      v = activate(act, v);
+      if (R != nullptr)
+        v += OUT_F16 ? __half2float(static_cast<const __half *>(R)[r * ldr + c])
+                     : static_cast<const float *>(R)[r * ldr + c];
+    }
     if constexpr (OUT_F16)
       reinterpret_cast<__half *>(C)[r * ldc + c] = __float2half_rn(v);
     else

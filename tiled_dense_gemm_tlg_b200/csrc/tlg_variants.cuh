@@ -20,7 +20,7 @@ struct LaunchState {
   int units = 0;
 };
 
-template <int CG, int TN, int STAGES, bool OUT_F16, bool BIAS_RELU, bool AT, bool BT, bool LSU>
+template <int CG, int TN, int STAGES, bool OUT_F16, int EK, bool AT, bool BT, bool LSU>
 struct Variant {
   static constexpr int NH = TN > 256 ? 2 : 1;  // MMA halves per tile
   static constexpr int BN = TN / NH;           // the MMA's N
@@ -56,7 +56,7 @@ struct Variant {
   // or the number of 2-CTA clusters the occupancy calculator admits.
   static tlg_status units(int dev, int sms, int *out) {
     static LaunchState state[kMaxDevices];
-    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH, AT, BT, LSU>;
+    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, EK, NH, AT, BT, LSU>;
     static std::mutex mutex;
     std::lock_guard<std::mutex> lock(mutex);
     LaunchState &st = state[dev];
@@ -92,7 +92,7 @@ struct Variant {
     fill_launch(&cfg, attr, s, overlap_prev);
     cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, BIAS_RELU, NH, AT, BT, LSU>, tmA, tmB, tmC,
+        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, EK, NH, AT, BT, LSU>, tmA, tmB, tmC,
         p);
     if (e != cudaSuccess) {
       cudaGetLastError();
@@ -116,13 +116,19 @@ constexpr int kNumVariants = 6;
     Variant<CG, TN, ST, F16, BR, AT, BT, L>::units,              \
         Variant<CG, TN, ST, F16, BR, AT, BT, L>::launch          \
   }
-#define TLG_VARIANT(CG, TN, ST, AT, BT, L)                                                     \
-  {                                                                                            \
-    TLG_FNS(CG, TN, ST, false, false, AT, BT, L), TLG_FNS(CG, TN, ST, true, false, AT, BT, L), \
-        TLG_FNS(CG, TN, ST, true, true, AT, BT, L)                                             \
+#define TLG_VARIANT(CG, TN, ST, AT, BT, L)                                              \
+  {                                                                                     \
+    TLG_FNS(CG, TN, ST, false, kEpiNone, AT, BT, L),                                    \
+        TLG_FNS(CG, TN, ST, true, kEpiNone, AT, BT, L),                                 \
+        TLG_FNS(CG, TN, ST, true, kEpiFused, AT, BT, L),                                \
+        TLG_FNS(CG, TN, ST, false, kEpiFused, AT, BT, L),                               \
+        TLG_FNS(CG, TN, ST, true, kEpiBiasRelu, AT, BT, L)                              \
   }
-#define TLG_NONE \
-  { VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr} }
+#define TLG_NONE                                                                          \
+  {                                                                                       \
+    VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr}, \
+        VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr}                        \
+  }
 #define TLG_LAYOUT(AT, BT)                                                                   \
   {                                                                                          \
     TLG_VARIANT(1, 64, 8, AT, BT, false), TLG_VARIANT(1, 128, 6, AT, BT, false),             \
@@ -137,10 +143,16 @@ constexpr int kNumVariants = 6;
   }
 
 
-// Tables of one operand layout: [variant, same order as the host's table][f32 | f16 | f16 bias+ReLU]
+// Output kinds of the launcher tables: plain fp32, plain fp16, the general
+// fused epilogue (bias / activation / residual) with an fp16 or an fp32 C, and
+// the bias + ReLU build with an fp16 C.
+constexpr int kKindF32 = 0, kKindF16 = 1, kKindF16Epi = 2, kKindF32Epi = 3, kKindF16BiasRelu = 4,
+              kNumKinds = 5;
+
+// Tables of one operand layout: [variant, same order as the host's table][output kind]
 struct LayoutTables {
-  VariantFns tma[kNumVariants][3];
-  VariantFns plain[kNumVariants][3];
+  VariantFns tma[kNumVariants][kNumKinds];
+  VariantFns plain[kNumVariants][kNumKinds];
 };
 
 // Defined by tlg_layout_{nn,nt,tn,tt}.cu.

@@ -15,6 +15,9 @@ GEMM on random fp16 inputs; page 3 "3.3" times a 1024x1024 matmul; page 4
   the ragged workload: ``randn * 0.25``; the bias: ``rand - 0.5``.
 * sampled output positions (for shapes whose full CPU reference is too slow)
   come from a second generator seeded with ``seed + 1``.
+* the residual of the general fused epilogue (page 4 "4.1": activation and
+  residual connection fused into the GEMM) comes from a third generator seeded
+  with ``seed + 2``: ``rand * 2 - 1`` cast to the output's type.
 """
 
 from __future__ import annotations
@@ -35,6 +38,15 @@ class Workload:
     out: str  # "f32" or "f16"
     bias_relu: bool
     sample: Optional[int] = None  # number of sampled output positions checked, None = all
+    # General fused epilogue C = act(A.B + bias) + R: the activation ("none",
+    # "relu" or "gelu"; None = not this epilogue), always with a bias, and
+    # whether a residual R in C's type is added.
+    act: Optional[str] = None
+    residual: bool = False
+
+    @property
+    def has_bias(self) -> bool:
+        return self.bias_relu or self.act is not None
 
     @property
     def flops(self) -> int:
@@ -46,10 +58,12 @@ class Workload:
 
     @property
     def algorithmic_bytes(self) -> int:
-        """Compulsory HBM bytes: A and B read once, C written once, bias read once."""
+        """Compulsory HBM bytes: A and B read once, C written once, bias and residual read once."""
         b = 2 * self.M * self.K + 2 * self.K * self.N + self.out_bytes * self.M * self.N
-        if self.bias_relu:
+        if self.has_bias:
             b += 2 * self.N
+        if self.residual:
+            b += self.out_bytes * self.M * self.N
         return b
 
 
@@ -65,6 +79,16 @@ WORKLOADS = {
     )
 }
 WORKLOAD_ORDER = list(WORKLOADS)
+
+# Fused-epilogue workloads beyond the five: bias + GELU + residual connection
+# at the bias+ReLU workload's size (a separate fp16 residual R, read once).
+EPILOGUE_WORKLOADS = {
+    w.name: w
+    for w in (
+        Workload("gemm_bias_gelu_residual_4096_f16", 4096, 4096, 4096, "uniform", "f16", False,
+                 sample=4096, act="gelu", residual=True),
+    )
+}
 
 
 def _draw(shape, dist: str, g: torch.Generator) -> torch.Tensor:
@@ -90,7 +114,15 @@ def make_operands(M: int, N: int, K: int, dist: str = "uniform", bias: bool = Fa
 
 
 def workload_operands(w: Workload, seed: int = 0):
-    return make_operands(w.M, w.N, w.K, w.dist, w.bias_relu, seed)
+    return make_operands(w.M, w.N, w.K, w.dist, w.has_bias, seed)
+
+
+def make_residual(M: int, N: int, out: str = "f16", seed: int = 0) -> torch.Tensor:
+    """A CPU residual ``R[M,N]`` in the output's type (``out`` "f16" or "f32"), entries in [-1, 1]."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed + 2)
+    x = torch.rand((M, N), generator=g, dtype=torch.float32) * 2.0 - 1.0
+    return x.to(torch.float16 if out == "f16" else torch.float32)
 
 
 def sample_positions(M: int, N: int, count: int, seed: int = 1):
