@@ -92,8 +92,77 @@ def nvsmi_id(dev) -> str:
         return str(dev.index or 0)
 
 
+class NvmlClockSampler:
+    """Polls the SM clock, its maximum, the clock-event (throttle) reasons and the power draw
+    through NVML every ~2 ms from a thread, and keeps the samples taken between mark_begin()
+    and mark_end() (the timed region).  Read-only queries: no GPU setting is touched."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, uuid: str):
+        import pynvml
+
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.samples = []  # (t, sm_mhz, reasons bitmask, power W)
+        self.t0 = self.t1 = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _poll(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((time.perf_counter(), sm, rs, pw))
+            except Exception:  # pragma: no cover - a failed query just loses a sample
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
+
+    def mark_begin(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def stop(self):
+        time.sleep(0.01)
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=2)
+        inside = [x for x in self.samples if self.t0 is not None and self.t1 is not None
+                  and self.t0 <= x[0] <= self.t1]
+        if not inside and self.samples and self.t0 is not None:
+            # a very short timed region: the samples nearest to it
+            inside = sorted(self.samples, key=lambda x: abs(x[0] - self.t0))[:3]
+        if not inside:
+            return None
+        mask = 0
+        for x in inside:
+            mask |= x[2]
+        reasons = sorted(name for name, const in self.REASONS
+                         if hasattr(self.nv, const) and mask & getattr(self.nv, const))
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside),
+                "power_w_median": statistics.median(x[3] for x in inside),
+                "window_ms": 1e3 * ((self.t1 or 0) - (self.t0 or 0)), "source": "nvml, 2 ms polling"}
+
+
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs
+    (fallback when NVML cannot be loaded; 100 ms sampling)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -117,6 +186,12 @@ class ClockSampler:
         self._thread = threading.Thread(target=self._read, daemon=True)
         self._thread.start()
         time.sleep(0.3)
+
+    def mark_begin(self):
+        pass
+
+    def mark_end(self):
+        pass
 
     def _read(self):
         for line in self.proc.stdout:
@@ -398,6 +473,13 @@ def main(argv=None):
         torch.cuda.synchronize(dev)
         return [s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)]
 
+    # The clock sampler starts before the warm-up, so the timed steps follow the warm-up
+    # directly (no idle gap in which the GPU clocks down).
+    try:
+        clocks = NvmlClockSampler(nvsmi_id(dev))
+    except Exception:
+        clocks = ClockSampler(nvsmi_id(dev))
+    clocks.start()
     for _ in range(args.warmup):
         flush.fill_(1.0)
         step()
@@ -406,11 +488,11 @@ def main(argv=None):
     if rc != 0:
         raise SystemExit(f"device error word {code:#x} during warm-up")
 
-    clocks = ClockSampler(nvsmi_id(dev))
-    clocks.start()
     barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.mark_begin()
     per_step_ms = timed(step, args.steps)
+    clocks.mark_end()
     barrier(world)
     clk = clocks.stop()
     gemm_ms = sum(per_step_ms)

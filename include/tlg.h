@@ -117,7 +117,9 @@ typedef enum tlg_epilogue { TLG_EPI_NONE = 0, TLG_EPI_BIAS_RELU = 1 } tlg_epilog
  *   stages      : depth of the shared-memory operand ring (fixed per tile shape)
  *   cta_group   : 1 (one SM per 128-row tile) or 2 (an SM pair per 256-row tile)
  *   raster_group: number of tile rows walked together for L2 reuse, 1..64
- *   max_ctas    : cap on resident CTAs (0 = one per SM)
+ *   max_ctas    : cap on resident CTAs (0 = one per SM, or as many 2-CTA
+ *                 clusters as the device can hold); tlg_choose_config
+ *                 reports the number of CTAs the launch would use
  *   split_k     : 0 or 1 = every tile whole; 2..16 = the tiles left over
  *                 after the last full wave are cut into that many k-slices
  *                 (needs a workspace).  The automatic choice does not split:

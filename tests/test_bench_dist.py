@@ -56,3 +56,24 @@ def test_single_rank_reductions_are_identity():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.job_throughput(1e12, 10, 1, 1000.0) == pytest.approx(10.0)  # 1e13 FLOP in 1 s
+
+
+def test_nvml_sampler_keeps_the_timed_window():
+    # The NVML sampler's summary on synthetic samples (no GPU, no NVML calls).
+    import types
+
+    import bench
+
+    fake = types.SimpleNamespace(nvmlClocksEventReasonSwPowerCap=0x4, nvmlClocksEventReasonHwSlowdown=0x8,
+                                 nvmlClocksEventReasonHwThermalSlowdown=0x40,
+                                 nvmlClocksEventReasonSwThermalSlowdown=0x20,
+                                 nvmlClocksEventReasonHwPowerBrakeSlowdown=0x80)
+    s = bench.NvmlClockSampler.__new__(bench.NvmlClockSampler)
+    s.nv, s.max_mhz, s._thread = fake, 1965, None
+    s._stop = bench.threading.Event()
+    s.samples = [(0.5, 1965, 0x0, 200.0), (1.1, 1500, 0x4, 990.0), (1.2, 1400, 0x4, 1000.0),
+                 (1.3, 1600, 0x0, 900.0), (2.5, 1965, 0x0, 150.0)]
+    s.t0, s.t1 = 1.0, 1.35
+    out = s.stop()
+    assert out["samples"] == 3 and out["sm_mhz"] == 1500 and out["reasons"] == ["sw_power_cap"]
+    assert out["sm_max_mhz"] == 1965 and out["power_w_median"] == 990.0

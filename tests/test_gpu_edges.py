@@ -223,9 +223,14 @@ def test_argument_errors(tlg, lib):
 
 
 def test_choose_config_matches_table(tlg):
+    props = torch.cuda.get_device_properties(0)
     for name, w in wl.WORKLOADS.items():
         c = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu)
-        assert c["block_n"] in (64, 128, 256) and c["stages"] >= 2
+        assert c["block_n"] in (64, 128, 256, 512) and c["stages"] >= 2
+        # the reported CTA count: whole groups, at most one CTA per SM
+        assert 0 < c["max_ctas"] <= props.multi_processor_count and c["max_ctas"] % c["cta_group"] == 0
+        # asking for exactly that configuration resolves to itself
+        assert tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.bias_relu, request=c) == c
 
 
 def test_timeout_path_reports_and_recovers(tlg):
