@@ -120,11 +120,14 @@ typedef enum tlg_epilogue { TLG_EPI_NONE = 0, TLG_EPI_BIAS_RELU = 1 } tlg_epilog
  *   max_ctas    : cap on resident CTAs (0 = one per SM, or as many 2-CTA
  *                 clusters as the device can hold); tlg_choose_config
  *                 reports the number of CTAs the launch would use
- *   split_k     : 0 or 1 = every tile whole; 2..16 = the tiles left over
- *                 after the last full wave are cut into that many k-slices
- *                 (needs a workspace).  The automatic choice does not split:
- *                 on a B200 under its power cap a split tail measured no
- *                 faster at 4096^3 and slower at 1024^3.
+ *   split_k     : 1 = every tile whole; 2..16 = the tiles left over after
+ *                 the last full wave are cut into that many k-slices (needs a
+ *                 workspace).  0 = automatic: every tile whole, or, when the
+ *                 call supplies a workspace large enough, a split tail of
+ *                 2..4 slices behind at least one whole wave where the cost
+ *                 model ranks it faster (measured on a B200: +4.5 % at
+ *                 4096^3 fp16 with split 2).  Calls without a workspace never
+ *                 split.
  *   overlap_prev: 1 = the kernel may begin its set-up (barriers, TMEM, tensor
  *                 maps) while the previous kernel in the stream is still
  *                 finishing (programmatic dependent launch); it reads and
@@ -303,7 +306,8 @@ tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
  * Resolve a configuration for this shape.  On input *config (never NULL)
  * holds the requested fields, zero meaning "choose for me" (all zero: the
  * automatic choice); on output it holds the configuration tlg_gemm_ex would
- * run, every field filled in.  TLG_ERR_UNSUPPORTED if the request names a
+ * run given a workspace of tlg_gemm_workspace_size() bytes, every field
+ * filled in.  TLG_ERR_UNSUPPORTED if the request names a
  * combination the library does not provide.  No kernel is launched; the only
  * CUDA calls read the current device's attributes.
  */

@@ -93,7 +93,8 @@ def test_forced_split_on_the_bias_relu_workload(tlg):
     cfg = {"cta_group": 2, "block_n": 256, "split_k": 2}
     nbytes = tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, "f16", True, cfg)
     assert nbytes > 4096
-    assert tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, "f16", True) == 0  # automatic: no split
+    # automatic: whole tiles, or (given the scratch) this same split of the partial last wave
+    assert tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, "f16", True) in (0, nbytes)
     A, B, bias = wl.workload_operands(w)
     ws = tlg.tlg_workspace(nbytes)
     C = tlg.tlg_gemm_ex(A.cuda(), B.cuda(), bias.cuda(), out="f16", config=cfg, workspace=ws)
@@ -121,3 +122,33 @@ def test_split_without_workspace_is_rejected_or_skipped(tlg):
 def test_no_device_error_after_split_runs(tlg):
     rc, code = tlg.tlg_device_error(clear=True)
     assert rc == 0 and code == 0, hex(code)
+
+
+def test_automatic_split_with_a_workspace(tlg):
+    # 256 pair tiles on 74 pairs leave a partial last wave; with a workspace the automatic
+    # choice splits that tail (and only then); the result is the forced split's, bit for bit.
+    M, N, K = 4096, 4096, 512
+    A, B, bias = wl.make_operands(M, N, K, "uniform", bias=True, seed=91)
+    auto = tlg.tlg_choose_config(M, N, K, "f16", True)
+    nbytes = tlg.tlg_gemm_workspace_size(M, N, K, "f16", True)
+    dA, dB, db = A.cuda(), B.cuda(), bias.cuda()
+    plain = tlg.tlg_gemm_bias_relu_f16(dA, dB, db)
+    if auto["split_k"] < 2:
+        assert nbytes == 0
+        pytest.skip(f"no split chosen on this device: {auto}")
+    assert nbytes > 0
+    ws = tlg.tlg_workspace(nbytes)
+    C = tlg.tlg_gemm_ex(dA, dB, db, out="f16", workspace=ws)
+    forced = tlg.tlg_gemm_ex(dA, dB, db, out="f16", config=auto, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(C, forced)
+    assert int(ws[:4096].count_nonzero()) == 0
+    rows, cols = wl.sample_positions(M, N, 4096, seed=92)
+    ref = oracle.gemm_at(A, B, rows.numpy(), cols.numpy(), bias=bias, relu=True)
+    for got in (C, plain):
+        ok, worst, idx = oracle.within_tolerance(got.double().cpu().numpy()[rows.numpy(), cols.numpy()], ref, "f16")
+        assert ok, f"worst err/bound {worst:.3g} at sample {idx}"
+    # without a workspace the same automatic call does not split (and still runs)
+    C2 = tlg.tlg_gemm_ex(dA, dB, db, out="f16")
+    torch.cuda.synchronize()
+    assert torch.equal(C2, plain)

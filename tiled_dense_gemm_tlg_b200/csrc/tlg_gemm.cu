@@ -220,25 +220,30 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
     if (r.max_ctas > 0) resident = std::max(1, std::min(resident, r.max_ctas / k.cta_group));
     const int64_t tile_m = 128 * k.cta_group;
     const int64_t tiles = ((M + tile_m - 1) / tile_m) * ((N + k.block_n - 1) / k.block_n);
-    // Automatic choice (split_k == 0) runs every tile whole: measured on a
-    // B200 the split tail gained nothing at 4096^3 (1353 vs 1349 TFLOP/s; under
-    // the 1000 W cap the SMs idle in a partial last wave let the busy ones
-    // clock higher) and lost at 1024^3, where its fix-up is exposed.
-    Schedule sch;
-    (void)ws_bytes;
-    if (!plan(tiles, resident, num_kb, r.split_k == 0 ? 1 : r.split_k, k.cta_group, k.block_n, &sch))
-      continue;
-    const double per_unit_tiles = static_cast<double>(tiles + sch.units - 1) / sch.units;
-    const double cost = (sch.cost + per_unit_tiles * k.exposed_kb) *
-                        static_cast<double>(tile_m * k.block_n) / (k.cta_group * k.eff);
-    if (!found || cost < best_cost * 0.999) {
-      found = true;
-      best_cost = cost;
-      out->idx = i;
-      out->sched = sch;
-      out->cfg.cta_group = k.cta_group;
-      out->cfg.block_n = k.block_n;
-      out->cfg.stages = k.stages;
+    // Automatic choice (split_k == 0): every tile whole, or, when the caller's
+    // workspace can hold it, a split tail of 2..4 k-slices if the model ranks
+    // it faster.  A split is only chosen behind at least one whole wave, whose
+    // tiles hide the partial sums' traffic: measured on a B200, split 2 at
+    // 4096^3 (3.46 waves) ran 4.5 % faster, while a split with no whole wave
+    // before it lost at 1024^3, where the fix-up is exposed.
+    const int split_lo = r.split_k == 0 ? 1 : r.split_k;
+    const int split_hi = r.split_k == 0 ? (ws_bytes > 0 ? 4 : 1) : r.split_k;
+    for (int split = split_lo; split <= split_hi; ++split) {
+      Schedule sch;
+      if (!plan(tiles, resident, num_kb, split, k.cta_group, k.block_n, &sch)) continue;
+      if (r.split_k == 0 && split > 1 && (sch.dp_tiles == 0 || sch.workspace > ws_bytes)) continue;
+      const double per_unit_tiles = static_cast<double>(tiles + sch.units - 1) / sch.units;
+      const double cost = (sch.cost + per_unit_tiles * k.exposed_kb) *
+                          static_cast<double>(tile_m * k.block_n) / (k.cta_group * k.eff);
+      if (!found || cost < best_cost * 0.999) {
+        found = true;
+        best_cost = cost;
+        out->idx = i;
+        out->sched = sch;
+        out->cfg.cta_group = k.cta_group;
+        out->cfg.block_n = k.block_n;
+        out->cfg.stages = k.stages;
+      }
     }
   }
   if (!shape_exists || !found) return TLG_ERR_UNSUPPORTED;
