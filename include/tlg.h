@@ -27,7 +27,14 @@
  *    C must not overlap A, B or the bias.
  *  - The call is asynchronous: it enqueues work on `stream` (a cudaStream_t;
  *    NULL means the legacy default stream) and returns.  Calls are
- *    stream-ordered and may be issued from several host threads.
+ *    stream-ordered and may be issued from several host threads and on
+ *    several streams at once.
+ *  - CUDA graphs: a call may be captured into a graph (stream capture) once
+ *    a call with the same kernel configuration has run eagerly on the device
+ *    (the first call sets the kernel's launch attributes).  The graph keeps
+ *    the pointers, sizes and tensor maps of the captured call; each replay
+ *    recomputes C from the buffers' current contents.  A split-K workspace
+ *    is left ready for the next replay.
  *  - The library allocates no device memory.
  *  - Alignment: every pointer must be aligned to its element (2 bytes for fp16
  *    data, 4 for an fp32 C), else TLG_ERR_ALIGNMENT.  The fast path loads and
