@@ -42,8 +42,10 @@
  *    row strides (lda*2, ldb*2, ldc*sizeof(out)) that are multiples of 16
  *    bytes; operands that break that rule are loaded by plain loads (several
  *    times slower) and such a C is written by plain stores.
- *  - Sizes: 0 <= M, N, K <= 2^31 - 257, and ceil(M/128)*ceil(N/64) below 2^31
- *    (larger sizes give TLG_ERR_UNSUPPORTED); lda >= K, ldb >= N, ldc >= N.
+ *  - Sizes: 0 <= M, N, K <= 2^31 - 257, and ceil(M/128)*ceil(N/64) below 2^31;
+ *    leading dimensions at most 2^36 elements and every matrix spanning less
+ *    than 2^60 bytes (larger sizes give TLG_ERR_UNSUPPORTED); lda >= K,
+ *    ldb >= N, ldc >= N.
  *    M == 0 or N == 0: nothing is written, TLG_OK.  K == 0: the empty sum is
  *    0, so C = 0 (bias variant: C = fp16(max(bias[col], 0)); tlg_gemm_fused:
  *    C = act(bias[col]) + residual).

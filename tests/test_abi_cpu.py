@@ -123,3 +123,24 @@ def test_fused_epilogue_host_side_rejections(lib_path):
     # empty shapes are fine with any valid descriptor
     assert lib.tlg_gemm_fused(0, 8, 8, 0, None, 8, 0, None, 8, ctypes.byref(E(None, 2, None, 0)), None, 8, 1,
                               None, None, 0, None) == tlg.TLG_OK
+
+
+def test_extent_overflow_is_rejected_on_the_host(lib_path):
+    import tiled_dense_gemm_tlg_b200 as tlg
+    lib = tlg.raw_library()
+    A = 1 << 20
+    # M * ldc * 4 bytes would pass 2^64 with these sizes: refused before any address arithmetic
+    assert lib.tlg_gemm_f16f32(2 ** 31 - 300, 8, 8, A, 8, A, 8, A * 4, 2 ** 36, None) == tlg.TLG_ERR_UNSUPPORTED
+    assert lib.tlg_gemm_f16f32(2 ** 30, 8, 8, A, 2 ** 36, A, 8, A * 4, 8, None) == tlg.TLG_ERR_UNSUPPORTED
+
+
+def test_binding_rejects_overlapping_views(lib_path):
+    import torch
+
+    import tiled_dense_gemm_tlg_b200 as tlg
+    row = torch.ones((1, 8), dtype=torch.float16)
+    B = torch.ones((8, 8), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        tlg.tlg_gemm_f16f32(row.expand(4, 8), B)  # row stride 0: four copies of one row
+    with pytest.raises(ValueError):
+        tlg.tlg_gemm_f16f32(B, torch.ones((8, 8), dtype=torch.float16).as_strided((8, 8), (4, 1)))

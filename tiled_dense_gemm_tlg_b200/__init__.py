@@ -125,6 +125,10 @@ def _mat(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be a 2-D tensor")
     if t.size(1) > 1 and t.stride(1) != 1:
         raise ValueError(f"{name} must be row-major (unit stride along its last dimension)")
+    if t.size(0) > 1 and t.stride(0) < t.size(1):
+        # a broadcast or overlapping view: its rows are not `stride(0)` elements apart in a
+        # buffer of rows x stride(0) elements, which is what the library would read
+        raise ValueError(f"{name} has overlapping rows (row stride {t.stride(0)} < {t.size(1)} columns)")
     return t.data_ptr(), max(t.stride(0), t.size(1))
 
 

@@ -352,6 +352,13 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, bool at, const void *A, i
   if (K > 0 && (misaligned(A, 2) || misaligned(B, 2))) return TLG_ERR_ALIGNMENT;
   if (ldc > (int64_t(1) << 36) || lda > (int64_t(1) << 36) || ldb > (int64_t(1) << 36))
     return TLG_ERR_UNSUPPORTED;
+  // Every matrix must span less than 2^60 bytes, so the extent arithmetic below
+  // cannot overflow (rows < 2^31 and ld <= 2^36 alone would allow 2^67).
+  auto spans = [](int64_t rows, int64_t ld, int64_t esz) {
+    return rows <= 1 || (rows - 1) <= ((int64_t(1) << 60) / esz) / ld;
+  };
+  if (!spans(M, ldc, osz) || (K > 0 && (!spans(at ? K : M, lda, 2) || !spans(bt ? N : K, ldb, 2))))
+    return TLG_ERR_UNSUPPORTED;
   uintptr_t c0, c1;
   extent(C, M, N, ldc, osz, &c0, &c1);
   if (K > 0) {
@@ -376,7 +383,7 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, bool at, const void *A, i
     // it); any other overlap with C would race.
     if (misaligned(e.R, static_cast<uintptr_t>(osz))) return TLG_ERR_ALIGNMENT;
     if (e.ldr < N) return TLG_ERR_INVALID_ARG;
-    if (e.ldr > (int64_t(1) << 36)) return TLG_ERR_UNSUPPORTED;
+    if (e.ldr > (int64_t(1) << 36) || !spans(M, e.ldr, osz)) return TLG_ERR_UNSUPPORTED;
     if (!(e.R == C && e.ldr == ldc)) {
       uintptr_t r0, r1;
       extent(e.R, M, N, e.ldr, osz, &r0, &r1);
