@@ -41,6 +41,7 @@ constexpr int kThreads = 32 * (2 + kEpiWarps);  // producer warp, MMA warp, epil
 constexpr int kLoaderWarps = 4;
 constexpr int kThreadsLsu = kThreads + 32 * kLoaderWarps;
 constexpr uint32_t kStageOutBytes = 32 * 128;   // one TMA store box: 32 rows x 128 bytes
+constexpr uint64_t kWaitPerKBlockNs = 20000;     // the epilogue's wait budget per k-block of a tile
 
 // Device error word (see tlg_device_error in tlg.h); internal linkage, so
 // every translation unit that includes this header has its own copy, and the
@@ -924,7 +925,12 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         if (w.tail < 0 && box_row0 < p.M && w.nb * kTileN < p.N)
           epi_prefetch<kPrefR>(p, box_row0 + lane, w.nb * kTileN, in);
       }
-      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.limit_ns, kRoleEpilogue,
+      // This wait spans the tile's whole main loop, so its limit grows with the
+      // tile's k-blocks (20 us each, far above a k-block's time on any built
+      // tile, the plain-load path included): a long K is not a stalled pipeline.
+      const uint64_t tile_limit_ns =
+          p.limit_ns + static_cast<uint64_t>(w.kb1 - w.kb0) * kWaitPerKBlockNs;
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, tile_limit_ns, kRoleEpilogue,
                      &g_device_error))
         break;
       tc_fence_after_sync();
