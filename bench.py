@@ -425,8 +425,13 @@ def main(argv=None):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     override = json.loads(args.config) if args.config else None
     kcfg = tlg.tlg_choose_config(w.M, w.N, w.K, w.out, w.has_bias, request=override)
-    # The split-K tail needs caller scratch; allocated once here, outside the timed region.
-    ws_bytes = tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, w.out, w.has_bias, override)
+    # The split-K tail and the aligned copies of operands TMA cannot describe need caller
+    # scratch; allocated once here, outside the timed region.
+    if args.ld_pad or at or bt:
+        ws_bytes = tlg.tlg_gemm_workspace_size_op(dA, dB, dC, args.layout[0], args.layout[1], w.out,
+                                                  config=override)
+    else:
+        ws_bytes = tlg.tlg_gemm_workspace_size(w.M, w.N, w.K, w.out, w.has_bias, override)
     ws = tlg.tlg_workspace(ws_bytes, device=dev) if ws_bytes > 0 else None
     fused = w.act is not None
     plain_name = ("tlg_gemm_fused" if fused else "tlg_gemm_bias_relu_f16" if w.bias_relu else
@@ -639,7 +644,8 @@ def main(argv=None):
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": dict(workload_config(w, kcfg), entry_point=entry, workspace_bytes=ws_bytes,
                        layout=args.layout, ld_pad=args.ld_pad,
-                       operand_path=("plain loads/stores (row strides not 16-byte multiples)"
+                       operand_path=(("aligned copies in the workspace, then TMA" if ws_bytes > 0
+                                      else "plain loads/stores") + " (row strides not 16-byte multiples)"
                                      if (args.ld_pad * 2) % 16 else "TMA")),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "plain_entry_point": plain,
         "gpu_launches": args.steps,

@@ -40,8 +40,10 @@
  *    data, 4 for an fp32 C), else TLG_ERR_ALIGNMENT.  The fast path loads and
  *    stores tiles with the TMA engine, which needs 16-byte aligned bases and
  *    row strides (lda*2, ldb*2, ldc*sizeof(out)) that are multiples of 16
- *    bytes; operands that break that rule are loaded by plain loads (several
- *    times slower) and such a C is written by plain stores.
+ *    bytes.  Operands that break that rule are copied into an aligned layout
+ *    when the call's workspace has room (tlg_gemm_workspace_size_op);
+ *    otherwise they are loaded by plain loads (several times slower) and such
+ *    a C is written by plain stores.
  *  - Sizes: 0 <= M, N, K <= 2^31 - 257, and ceil(M/128)*ceil(N/64) below 2^31;
  *    leading dimensions at most 2^36 elements and every matrix spanning less
  *    than 2^60 bytes (larger sizes give TLG_ERR_UNSUPPORTED); lda >= K,
@@ -310,6 +312,30 @@ tlg_status tlg_gemm_fused(int64_t M, int64_t N, int64_t K,
 tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
                                    tlg_epilogue epilogue, const tlg_config *config,
                                    size_t *bytes);
+
+/*
+ * Workspace bytes for a call with these operands (tlg_gemm_ex, tlg_gemm_op or
+ * tlg_gemm_fused with the same sizes, layouts, pointers and strides):
+ * the split-K scratch of the configuration (NULL = automatic), plus room for
+ * aligned copies of the matrices TMA cannot describe (a base address or row
+ * stride not a multiple of 16 bytes).
+ *
+ * Given that much workspace, a call copies each such A or B into an aligned
+ * layout in the workspace first and runs the TMA path on the copies; such a
+ * C is produced in the workspace and copied out at the end.  Each copy moves
+ * every byte once, so a call with odd strides then runs near the speed of
+ * an aligned one instead of on the plain-load path.  With less workspace the
+ * call still succeeds on the plain-load path (A and B copies are made only
+ * when both fit; a C copy when it fits after them).  The copies never touch
+ * the workspace's first 4 KB (the split-K counters).  0 when every matrix is
+ * aligned and no split is chosen.  Only host-side checks and device-attribute
+ * queries run; nothing is launched.
+ */
+tlg_status tlg_gemm_workspace_size_op(int64_t M, int64_t N, int64_t K,
+                                      tlg_op op_a, const void *A, int64_t lda,
+                                      tlg_op op_b, const void *B, int64_t ldb,
+                                      const void *C, int64_t ldc, tlg_out out,
+                                      const tlg_config *config, size_t *bytes);
 
 /*
  * Resolve a configuration for this shape.  On input *config (never NULL)

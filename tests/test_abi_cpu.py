@@ -144,3 +144,16 @@ def test_binding_rejects_overlapping_views(lib_path):
         tlg.tlg_gemm_f16f32(row.expand(4, 8), B)  # row stride 0: four copies of one row
     with pytest.raises(ValueError):
         tlg.tlg_gemm_f16f32(B, torch.ones((8, 8), dtype=torch.float16).as_strided((8, 8), (4, 1)))
+
+
+def test_workspace_size_op_host_checks(lib_path):
+    import tiled_dense_gemm_tlg_b200 as tlg
+    lib = tlg.raw_library()
+    A = 1 << 20
+    n = ctypes.c_size_t(7)
+    assert lib.tlg_gemm_workspace_size_op(8, 8, 8, 0, A, 8, 0, A, 8, A * 2, 8, 1, None, None) == tlg.TLG_ERR_INVALID_ARG
+    assert lib.tlg_gemm_workspace_size_op(8, 8, 8, 3, A, 8, 0, A, 8, A * 2, 8, 1, None, ctypes.byref(n)) == tlg.TLG_ERR_INVALID_ARG
+    assert n.value == 0
+    assert lib.tlg_gemm_workspace_size_op(8, 8, 8, 0, A, 7, 0, A, 8, A * 2, 8, 1, None, ctypes.byref(n)) == tlg.TLG_ERR_INVALID_ARG
+    assert lib.tlg_gemm_workspace_size_op(0, 8, 8, 0, None, 8, 0, None, 8, None, 8, 1, None, ctypes.byref(n)) == tlg.TLG_OK
+    assert n.value == 0

@@ -1,0 +1,125 @@
+"""Operands the TMA unit cannot describe, with a workspace large enough for aligned copies
+(tlg_gemm_workspace_size_op): the call copies such an A or B into the workspace, runs the TMA
+path on the copies, and produces such a C in the workspace and copies it out.  Every case is
+checked against the CPU oracle, with NaN guard bands around each caller matrix, and the
+workspace's split-K counters must be left zero."""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tlg_workloads as wl
+from test_gpu_unaligned import Raw
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tlg():
+    import tiled_dense_gemm_tlg_b200 as t
+    return t
+
+
+def call(tlg, A, B, bias, out, ld_extra, offsets=(0, 0, 0), op=("N", "N"), cfg=None, ws_mode="full",
+         act=None, residual=None, inplace=False):
+    """One call on raw buffers; ws_mode: "full" (the size query's bytes), "split" (only the
+    split scratch: copies do not fit) or "none"."""
+    lib = tlg.raw_library()
+    at, bt = op[0] == "T", op[1] == "T"
+    M, K = A.shape
+    N = B.shape[1]
+    sa = A.t().contiguous() if at else A
+    sb = B.t().contiguous() if bt else B
+    ra = Raw(sa, sa.shape[0], sa.shape[1], sa.shape[1] + ld_extra[0], torch.float16, offsets[0])
+    rb = Raw(sb, sb.shape[0], sb.shape[1], sb.shape[1] + ld_extra[1], torch.float16, offsets[1])
+    odt = torch.float32 if out == "f32" else torch.float16
+    rc_ = Raw(residual if inplace else None, M, N, N + ld_extra[2], odt, offsets[2])
+    dbias = bias.cuda() if bias is not None else None
+    c = tlg.tlg_config(**cfg) if cfg else None
+    o = tlg.TLG_OUT_F32 if out == "f32" else tlg.TLG_OUT_F16
+    full = ctypes.c_size_t(0)
+    rcq = lib.tlg_gemm_workspace_size_op(M, N, K, int(at), ra.ptr(), ra.ld, int(bt), rb.ptr(), rb.ld, rc_.ptr(),
+                                         rc_.ld, o, ctypes.byref(c) if c else None, ctypes.byref(full))
+    assert rcq == 0, tlg.tlg_status_string(rcq)
+    split_only = tlg.tlg_gemm_workspace_size(M, N, K, out, bias is not None, cfg)
+    nbytes = {"full": full.value, "split": split_only, "none": 0}[ws_mode]
+    ws = tlg.tlg_workspace(nbytes) if nbytes else None
+    epi = tlg.tlg_fused_epilogue(dbias.data_ptr() if dbias is not None else None,
+                                 {None: 0, "relu": 1, "gelu": 2}[act], None, 0)
+    if inplace:
+        epi.residual, epi.ldr = rc_.ptr(), rc_.ld
+    rc = lib.tlg_gemm_fused(M, N, K, int(at), ra.ptr(), ra.ld, int(bt), rb.ptr(), rb.ld, ctypes.byref(epi),
+                            rc_.ptr(), rc_.ld, o, ctypes.byref(c) if c else None,
+                            ws.data_ptr() if ws is not None else None, nbytes,
+                            int(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, tlg.tlg_status_string(rc)
+    torch.cuda.synchronize()
+    assert all(r.guard_ok() for r in (ra, rb, rc_)), "guard band changed"
+    if ws is not None:
+        assert int(ws[:4096].count_nonzero()) == 0, "split-K counters left non-zero"
+    return rc_.matrix().double().cpu().numpy(), full.value
+
+
+@pytest.mark.parametrize("out", ["f16", "f32"])
+@pytest.mark.parametrize("which", ["A", "B", "C", "AB", "ABC"])
+@pytest.mark.parametrize("ws_mode", ["full", "split", "none"])
+def test_copies_or_plain_loads(tlg, which, out, ws_mode):
+    M, N, K = 300, 264, 200
+    A, B, bias = wl.make_operands(M, N, K, "uniform", bias=True, seed=401)
+    ex = (1 if "A" in which else 8, 1 if "B" in which else 8, 1 if "C" in which else 16 // (4 if out == "f32" else 2))
+    offs = (1 if "A" in which else 0, 3 if "B" in which else 0, 1 if "C" in which else 0)
+    got, full = call(tlg, A, B, bias, out, ex, offs, ws_mode=ws_mode, act="relu")
+    assert full > 0
+    ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B, bias=bias, relu=True), out)
+    assert ok, (worst, idx)
+
+
+@pytest.mark.parametrize("op", [("T", "N"), ("N", "T"), ("T", "T")], ids=lambda o: o[0] + o[1])
+def test_copies_of_transposed_operands(tlg, op):
+    M, N, K = 260, 300, 136
+    A, B, _ = wl.make_operands(M, N, K, "normal025", seed=402)
+    got, _ = call(tlg, A, B, None, "f32", (3, 5, 1), (1, 1, 1), op=op)
+    ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B), "f32")
+    assert ok, (worst, idx)
+
+
+def test_copy_of_c_with_in_place_residual(tlg):
+    # R == C, both unaligned: the kernel reads R from the caller's C and writes the aligned copy,
+    # which is then copied over C
+    M, N, K = 300, 264, 200
+    A, B, bias = wl.make_operands(M, N, K, "uniform", bias=True, seed=403)
+    R = wl.make_residual(M, N, "f16", seed=403)
+    got, _ = call(tlg, A, B, bias, "f16", (1, 1, 1), (1, 1, 1), act="gelu", residual=R, inplace=True)
+    ok, worst, idx = oracle.within_tolerance(got, oracle.gemm_fused(A, B, bias=bias, act="gelu", residual=R), "f16")
+    assert ok, (worst, idx)
+
+
+def test_copies_with_a_forced_split(tlg):
+    M, N, K = 1024, 768, 1024
+    A, B, bias = wl.make_operands(M, N, K, "uniform", bias=True, seed=404)
+    cfg = {"cta_group": 2, "block_n": 256, "split_k": 4}
+    got, full = call(tlg, A, B, bias, "f16", (1, 1, 1), (1, 1, 1), cfg=cfg, act="relu")
+    assert full > tlg.tlg_gemm_workspace_size(M, N, K, "f16", True, cfg)
+    ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B, bias=bias, relu=True), "f16")
+    assert ok, (worst, idx)
+
+
+def test_integer_inputs_bit_exact_through_copies(tlg):
+    M, N, K = 700, 520, 1000
+    A, B, _ = wl.integer_operands(M, N, K, seed=405)
+    got, _ = call(tlg, A, B, None, "f32", (1, 1, 1), (1, 1, 1))
+    assert np.array_equal(got, oracle.gemm(A, B))
+
+
+def test_size_query_for_aligned_operands_is_the_split_scratch(tlg):
+    M = N = K = 4096
+    A = torch.empty((M, K), dtype=torch.float16, device="cuda")
+    B = torch.empty((K, N), dtype=torch.float16, device="cuda")
+    C = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    assert tlg.tlg_gemm_workspace_size_op(A, B, C) == tlg.tlg_gemm_workspace_size(M, N, K, "f16", False)
+    Ao = torch.empty((M, K + 1), dtype=torch.float16, device="cuda")[:, :K]
+    more = tlg.tlg_gemm_workspace_size_op(Ao, B, C)
+    assert more >= tlg.tlg_gemm_workspace_size(M, N, K, "f16", False) + M * K * 2

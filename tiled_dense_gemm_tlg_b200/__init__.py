@@ -47,7 +47,7 @@ TLG_ACT_NONE, TLG_ACT_RELU, TLG_ACT_GELU = 0, 1, 2
 _ACT = {"none": TLG_ACT_NONE, "relu": TLG_ACT_RELU, "gelu": TLG_ACT_GELU}
 
 EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-            "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
+            "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_gemm_workspace_size_op", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
             "tlg_version")
 
 
@@ -81,6 +81,8 @@ _lib.tlg_gemm_ex_noalloc.argtypes = [_i64, _i64, _i64, _p, _i64, _p, _i64, _p, _
                                      ctypes.POINTER(tlg_config), _p]
 _lib.tlg_gemm_workspace_size.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config),
                                          ctypes.POINTER(_sz)]
+_lib.tlg_gemm_workspace_size_op.argtypes = [_i64, _i64, _i64, _i32, _p, _i64, _i32, _p, _i64, _p, _i64, _i32,
+                                            ctypes.POINTER(tlg_config), ctypes.POINTER(_sz)]
 _lib.tlg_choose_config.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(tlg_config)]
 _lib.tlg_device_error.argtypes = [_i32, ctypes.POINTER(ctypes.c_uint32)]
 _lib.tlg_selftest_timeout.argtypes = [ctypes.c_uint32, _p]
@@ -88,7 +90,7 @@ _lib.tlg_status_string.argtypes = [_i32]
 _lib.tlg_status_string.restype = ctypes.c_char_p
 _lib.tlg_version.restype = ctypes.c_int32
 for _name in ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-              "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
+              "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_gemm_workspace_size_op", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout"):
     getattr(_lib, _name).restype = _i32
 
 
@@ -311,6 +313,31 @@ def tlg_gemm_workspace_size(M: int, N: int, K: int, out: str = "f32", bias_relu:
                                         TLG_EPI_BIAS_RELU if bias_relu else TLG_EPI_NONE,
                                         ctypes.byref(cfg) if cfg is not None else None, ctypes.byref(n)),
            "tlg_gemm_workspace_size")
+    return int(n.value)
+
+
+def tlg_gemm_workspace_size_op(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor | None = None,
+                               op_a: str = "N", op_b: str = "N", out: str = "f16",
+                               config: dict | None = None) -> int:
+    """Workspace bytes for a call on these operands: the split-K scratch plus aligned copies of
+    the matrices TMA cannot describe (see tlg.h).  C = None assumes an aligned C."""
+    at, bt = op_a.upper() == "T", op_b.upper() == "T"
+    M, K = (A.shape[1], A.shape[0]) if at else tuple(A.shape)
+    N = B.shape[0] if bt else B.shape[1]
+    pa, lda = _mat(A, "A")
+    pb, ldb = _mat(B, "B")
+    esz = 4 if out == "f32" else 2
+    if C is None:
+        pc, ldc = 1 << 20, ((N * esz + 15) // 16 * 16) // esz  # a stand-in aligned C
+    else:
+        pc, ldc = _mat(C, "C")
+    cfg = tlg_config(**{k: int(v) for k, v in config.items()}) if config else None
+    n = ctypes.c_size_t(0)
+    _check(_lib.tlg_gemm_workspace_size_op(M, N, K, TLG_OP_T if at else TLG_OP_N, pa, lda,
+                                           TLG_OP_T if bt else TLG_OP_N, pb, ldb, pc, ldc,
+                                           TLG_OUT_F32 if out == "f32" else TLG_OUT_F16,
+                                           ctypes.byref(cfg) if cfg is not None else None, ctypes.byref(n)),
+           "tlg_gemm_workspace_size_op")
     return int(n.value)
 
 

@@ -326,6 +326,113 @@ tlg_status launch_fill(void *C, int64_t ldc, const Epi &e, int M, int N, cudaStr
   return TLG_OK;
 }
 
+// ---------------------------------------------------------------- aligned copies
+//
+// Operands the TMA unit cannot describe (a base or row stride off 16 bytes) are
+// copied, when the call's workspace has room, into an aligned layout in the
+// workspace; the GEMM then runs its TMA path on the copies.  A C that TMA cannot
+// store is produced in the workspace and copied out.  Both copies are
+// memory-bound and move each byte once.
+
+constexpr size_t kCopyAlign = 256;
+
+size_t round_up_sz(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// An aligned copy of a rows x cols matrix of esz-byte elements: rows of
+// round_up(cols * esz, 16) bytes.
+size_t aligned_copy_bytes(int64_t rows, int64_t cols, int64_t esz) {
+  return round_up_sz(static_cast<size_t>(rows) * round_up_sz(static_cast<size_t>(cols * esz), 16),
+                     kCopyAlign);
+}
+
+// dst <- src for a rows x cols matrix of T, row strides in elements.
+// Consecutive lanes move consecutive elements of a row, so every warp access
+// is contiguous on both sides whatever the two matrices' alignments.  Each
+// thread keeps kCopyPer loads in flight before its stores: with 2-byte
+// elements, 4 per thread held about a third of the bytes in flight that HBM
+// latency needs at full bandwidth (measured ~2.3 TB/s), so a thread moves 16.
+constexpr int kCopyPer = 16;
+constexpr int kCopyThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kCopyThreads)
+    copy_2d_kernel(const T *__restrict__ src, int64_t src_ld, T *__restrict__ dst, int64_t dst_ld,
+                   int64_t rows, int64_t cols) {
+  const int64_t step = static_cast<int64_t>(kCopyPer) * kCopyThreads;
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+    const T *s = src + r * src_ld;
+    T *d = dst + r * dst_ld;
+    for (int64_t c0 = blockIdx.x * step; c0 < cols; c0 += static_cast<int64_t>(gridDim.x) * step) {
+      T v[kCopyPer];
+#pragma unroll
+      for (int k = 0; k < kCopyPer; ++k) {
+        const int64_t c = c0 + k * kCopyThreads + threadIdx.x;
+        if (c < cols) v[k] = s[c];
+      }
+#pragma unroll
+      for (int k = 0; k < kCopyPer; ++k) {
+        const int64_t c = c0 + k * kCopyThreads + threadIdx.x;
+        if (c < cols) d[c] = v[k];
+      }
+    }
+  }
+}
+
+dim3 copy_grid(int64_t rows, int64_t cols) {
+  const int64_t per_block = static_cast<int64_t>(kCopyPer) * kCopyThreads;
+  const int64_t gx = std::min<int64_t>((cols + per_block - 1) / per_block, 64);
+  const int64_t gy = std::min<int64_t>(rows, 16384);
+  return dim3(static_cast<unsigned>(std::max<int64_t>(gx, 1)),
+              static_cast<unsigned>(std::max<int64_t>(gy, 1)), 1);
+}
+
+// Aligned row stride, in elements, of a copy of a matrix with `cols` columns.
+int64_t aligned_ld(int64_t cols, int64_t esz) {
+  return static_cast<int64_t>(round_up_sz(static_cast<size_t>(cols * esz), 16)) / esz;
+}
+
+tlg_status launch_copy(const void *src, int64_t src_ld, void *dst, int64_t dst_ld, int64_t rows,
+                       int64_t cols, int64_t esz, cudaStream_t s) {
+  const dim3 grid = copy_grid(rows, cols);
+  if (esz == 2)
+    copy_2d_kernel<unsigned short><<<grid, kCopyThreads, 0, s>>>(static_cast<const unsigned short *>(src),
+                                                        src_ld, static_cast<unsigned short *>(dst),
+                                                        dst_ld, rows, cols);
+  else
+    copy_2d_kernel<uint32_t><<<grid, kCopyThreads, 0, s>>>(static_cast<const uint32_t *>(src), src_ld,
+                                                  static_cast<uint32_t *>(dst), dst_ld, rows, cols);
+  if (cudaPeekAtLastError() != cudaSuccess) {
+    cudaGetLastError();
+    return TLG_ERR_CUDA;
+  }
+  return TLG_OK;
+}
+
+// Which of the call's matrices TMA cannot describe, and the workspace their
+// aligned copies take.
+struct CopyPlan {
+  bool a = false, b = false, c = false;
+  size_t a_bytes = 0, b_bytes = 0, c_bytes = 0;
+  size_t ab_bytes() const { return a_bytes + b_bytes; }
+};
+
+CopyPlan copy_plan(int64_t M, int64_t N, int64_t K, bool at, const void *A, int64_t lda, bool bt,
+                   const void *B, int64_t ldb, const void *C, int64_t ldc, int64_t osz) {
+  CopyPlan cp;
+  auto tma_ok = [](const void *q, int64_t ld, int64_t esz) {
+    return (reinterpret_cast<uintptr_t>(q) & 15u) == 0 && (ld * esz) % 16 == 0;
+  };
+  if (K > 0) {
+    cp.a = !tma_ok(A, lda, 2);
+    cp.b = !tma_ok(B, ldb, 2);
+    if (cp.a) cp.a_bytes = aligned_copy_bytes(at ? K : M, at ? M : K, 2);
+    if (cp.b) cp.b_bytes = aligned_copy_bytes(bt ? N : K, bt ? K : N, 2);
+  }
+  cp.c = !tma_ok(C, ldc, osz);
+  if (cp.c) cp.c_bytes = aligned_copy_bytes(M, N, osz);
+  return cp;
+}
+
 // Host-only argument checks shared by every entry point; nothing here touches the GPU.
 // at / bt: A stored K x M (lda >= M), B stored N x K (ldb >= K), the product
 // using their transposes.
@@ -450,14 +557,58 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
                               ? kEpiBiasRelu
                               : kEpiFused;
 
-  // TMA needs 16-byte aligned bases and row strides.
-  const bool plain = !(aligned16(A) && aligned16(B) && (lda * 2) % 16 == 0 && (ldb * 2) % 16 == 0);
-  const bool c_plain = !(aligned16(C) && (ldc * osz) % 16 == 0);
+  // TMA needs 16-byte aligned bases and row strides.  Operands that break
+  // that rule are copied into an aligned layout in the workspace when it has
+  // room (after the split-K scratch, never over its counters); otherwise A and
+  // B go through the plain-load warps and C through plain stores.
+  const CopyPlan cp = copy_plan(M, N, K, at, A, lda, bt, B, ldb, C, ldc, osz);
+  bool copy_ab = false, copy_c = false;
   Resolved rv;
-  const tlg_status rs =
-      resolve(dev, info.sm_count, M, N, K, f16, ek, at, bt, plain, req, ws_bytes, &rv);
+  tlg_status rs = TLG_ERR_UNSUPPORTED;
+  size_t copy_base = 0;
+  if ((cp.a || cp.b) && ws_bytes >= kCounterBytes + cp.ab_bytes()) {
+    // the TMA path with copies of A and/or B, split scratch from what is left
+    rs = resolve(dev, info.sm_count, M, N, K, f16, ek, at, bt, false, req,
+                 ws_bytes - kCounterBytes - cp.ab_bytes(), &rv);
+    if (rs == TLG_OK) {
+      copy_ab = true;
+      copy_base = round_up_sz(std::max<size_t>(rv.sched.workspace, kCounterBytes), kCopyAlign);
+      if (copy_base + cp.ab_bytes() > ws_bytes) copy_ab = false;
+    }
+  }
+  const bool plain = (cp.a || cp.b) && !copy_ab;
+  if (!copy_ab) {
+    rs = resolve(dev, info.sm_count, M, N, K, f16, ek, at, bt, plain, req, ws_bytes, &rv);
+    copy_base = round_up_sz(std::max<size_t>(rv.sched.workspace, kCounterBytes), kCopyAlign);
+  }
   if (rs != TLG_OK) return rs;
   if (rv.sched.workspace > ws_bytes) return TLG_ERR_INVALID_ARG;  // a forced split needs scratch
+  const size_t c_off = copy_base + (copy_ab ? cp.ab_bytes() : 0);
+  if (cp.c && ws != nullptr && c_off + cp.c_bytes <= ws_bytes) copy_c = true;
+  const bool c_plain = cp.c && !copy_c;
+  char *wsb = static_cast<char *>(ws);
+  const void *A_use = A, *B_use = B;
+  int64_t lda_use = lda, ldb_use = ldb;
+  if (copy_ab) {
+    size_t off = copy_base;
+    if (cp.a) {
+      const int64_t rows = at ? K : M, cols = at ? M : K;
+      lda_use = aligned_ld(cols, 2);
+      const tlg_status cs = launch_copy(A, lda, wsb + off, lda_use, rows, cols, 2, s);
+      if (cs != TLG_OK) return cs;
+      A_use = wsb + off;
+      off += cp.a_bytes;
+    }
+    if (cp.b) {
+      const int64_t rows = bt ? N : K, cols = bt ? K : N;
+      ldb_use = aligned_ld(cols, 2);
+      const tlg_status cs = launch_copy(B, ldb, wsb + off, ldb_use, rows, cols, 2, s);
+      if (cs != TLG_OK) return cs;
+      B_use = wsb + off;
+    }
+  }
+  void *C_use = copy_c ? static_cast<void *>(wsb + c_off) : C;
+  const int64_t ldc_use = copy_c ? aligned_ld(N, osz) : ldc;
 
   // Boxes (inner x outer, elements): A 64 k x 128 rows, or 64 m x 64 k when
   // stored transposed; B 64 n x 64 k, or 64 k x (columns per CTA) when stored
@@ -469,21 +620,21 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   const uint32_t b_rows_per_cta =
       static_cast<uint32_t>((rv.cfg.block_n > 256 ? 256 : rv.cfg.block_n) / rv.cfg.cta_group);
   if (!plain) {
-    const bool a_ok = at ? encode_2d(&tmA, h16, A, uint64_t(M), uint64_t(K), uint64_t(lda) * 2, 64, kBK)
-                         : encode_2d(&tmA, h16, A, uint64_t(K), uint64_t(M), uint64_t(lda) * 2, kBK, kBM);
-    const bool b_ok = bt ? encode_2d(&tmB, h16, B, uint64_t(K), uint64_t(N), uint64_t(ldb) * 2, kBK,
+    const bool a_ok = at ? encode_2d(&tmA, h16, A_use, uint64_t(M), uint64_t(K), uint64_t(lda_use) * 2, 64, kBK)
+                         : encode_2d(&tmA, h16, A_use, uint64_t(K), uint64_t(M), uint64_t(lda_use) * 2, kBK, kBM);
+    const bool b_ok = bt ? encode_2d(&tmB, h16, B_use, uint64_t(K), uint64_t(N), uint64_t(ldb_use) * 2, kBK,
                                      b_rows_per_cta)
-                         : encode_2d(&tmB, h16, B, uint64_t(N), uint64_t(K), uint64_t(ldb) * 2, 64, kBK);
+                         : encode_2d(&tmB, h16, B_use, uint64_t(N), uint64_t(K), uint64_t(ldb_use) * 2, 64, kBK);
     if (!a_ok || !b_ok) return TLG_ERR_CUDA;
   }
-  if (!c_plain && !encode_2d(&tmC, c_type, C, uint64_t(N), uint64_t(M), uint64_t(ldc) * osz,
+  if (!c_plain && !encode_2d(&tmC, c_type, C_use, uint64_t(N), uint64_t(M), uint64_t(ldc_use) * osz,
                              uint32_t(128 / osz), 32))
     return TLG_ERR_CUDA;
 
   GemmParams p;
   p.bias = static_cast<const __half *>(bias);
-  p.C = C;
-  p.ldc = ldc;
+  p.C = C_use;
+  p.ldc = ldc_use;
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
@@ -496,18 +647,20 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   p.counters = static_cast<uint32_t *>(ws);
   p.ws = ws != nullptr ? reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes)
                        : nullptr;
-  p.A = static_cast<const __half *>(A);
-  p.B = static_cast<const __half *>(B);
-  p.lda = lda;
-  p.ldb = ldb;
+  p.A = static_cast<const __half *>(A_use);
+  p.B = static_cast<const __half *>(B_use);
+  p.lda = lda_use;
+  p.ldb = ldb_use;
   p.c_plain = c_plain ? 1 : 0;
   p.bias_aligned = (bias != nullptr && aligned16(bias)) ? 1 : 0;
   p.act = e.act;
   p.R = e.R;
   p.ldr = e.ldr;
   p.r_vec = (e.R != nullptr && aligned16(e.R) && (e.ldr * osz) % 16 == 0) ? 1 : 0;
-  return fns_for(rv.idx, f16, ek, at, bt, plain)
-      .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
+  const tlg_status ls = fns_for(rv.idx, f16, ek, at, bt, plain)
+                             .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
+  if (ls != TLG_OK || !copy_c) return ls;
+  return launch_copy(C_use, aligned_ld(N, osz), C, ldc, M, N, osz, s);
 }
 
 // ---------------------------------------------------------------- allocation-free scratch
@@ -693,6 +846,36 @@ tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
   const tlg_status rs = resolve_public(M, N, K, out, epilogue, config, SIZE_MAX, &rv);
   if (rs != TLG_OK) return rs;
   *bytes = rv.sched.workspace;
+  return TLG_OK;
+}
+
+tlg_status tlg_gemm_workspace_size_op(int64_t M, int64_t N, int64_t K, tlg_op op_a,
+                                      const void *A, int64_t lda, tlg_op op_b, const void *B,
+                                      int64_t ldb, const void *C, int64_t ldc, tlg_out out,
+                                      const tlg_config *config, size_t *bytes) {
+  if (bytes == nullptr) return TLG_ERR_INVALID_ARG;
+  *bytes = 0;
+  if ((op_a != TLG_OP_N && op_a != TLG_OP_T) || (op_b != TLG_OP_N && op_b != TLG_OP_T))
+    return TLG_ERR_INVALID_ARG;
+  const bool at = op_a == TLG_OP_T, bt = op_b == TLG_OP_T;
+  const tlg_status hs = check_args(M, N, K, at, A, lda, bt, B, ldb, Epi{}, C, ldc, out);
+  if (hs != TLG_OK || M == 0 || N == 0 || K == 0) return hs;
+  const int64_t osz = out == TLG_OUT_F32 ? 4 : 2;
+  const CopyPlan cp = copy_plan(M, N, K, at, A, lda, bt, B, ldb, C, ldc, osz);
+  int dev = 0;
+  DeviceInfo info;
+  const tlg_status ds = current_device(&dev, &info);
+  if (ds != TLG_OK) return ds;
+  Resolved rv;
+  const tlg_status rs = resolve(dev, info.sm_count, M, N, K, out == TLG_OUT_F16, kEpiNone, at, bt,
+                                false, config, SIZE_MAX, &rv);
+  if (rs != TLG_OK) return rs;
+  if (!cp.a && !cp.b && !cp.c) {
+    *bytes = rv.sched.workspace;
+    return TLG_OK;
+  }
+  *bytes = round_up_sz(std::max<size_t>(rv.sched.workspace, kCounterBytes), kCopyAlign) +
+           cp.ab_bytes() + cp.c_bytes;
   return TLG_OK;
 }
 
