@@ -17,8 +17,10 @@ Functions and the passages they follow:
   (xdnf.cn/news/333523) section 4.2).
 * ``gemm_at`` -- the same value at selected (row, col) positions.
 * ``gemm_fused`` / ``gemm_at_fused`` -- act(A.B + bias[col]) + R[row, col] with
-  act in {none, relu, gelu} ("domestic-GPU TileLang adoption" section 4.1:
-  activation and residual fused into the operator; GELU in its exact erf form).
+  act in {none, relu, gelu, silu, gelu_tanh} ("domestic-GPU TileLang adoption"
+  section 4.1: activation and residual fused into the operator; the pages give
+  no formulas, so each activation is its standard definition: GELU in its exact
+  erf form, SiLU x*sigmoid(x), and the tanh form of GELU).
 
 Every function is pinned by tests/test_oracle_pins.py; none is parity unpinned.
 """
@@ -181,7 +183,7 @@ def gemm_at(A, B, rows, cols, bias=None, relu: bool = False, threads: int | None
     return out
 
 
-ACT = {"none": 0, "relu": 1, "gelu": 2}
+ACT = {"none": 0, "relu": 1, "gelu": 2, "silu": 3, "gelu_tanh": 4}
 
 
 def activation(x: float, act: str) -> float:

@@ -97,14 +97,34 @@ void oracle_f16_encode_array(const double *x, uint16_t *out, int64_t n)
 }
 
 /* Activation codes shared by the fused routines below. */
-enum { ORACLE_ACT_NONE = 0, ORACLE_ACT_RELU = 1, ORACLE_ACT_GELU = 2 };
+enum {
+    ORACLE_ACT_NONE = 0,
+    ORACLE_ACT_RELU = 1,
+    ORACLE_ACT_GELU = 2,
+    ORACLE_ACT_SILU = 3,
+    ORACLE_ACT_GELU_TANH = 4
+};
 
+/*
+ * The activations by their standard definitions (the pages name activation
+ * fusion but print no formulas):
+ *   ReLU  max(x, 0)
+ *   GELU  x * Phi(x) = x/2 * (1 + erf(x / sqrt 2))
+ *   SiLU  x * sigmoid(x) = x / (1 + exp(-x))
+ *   GELU, tanh form  x/2 * (1 + tanh(sqrt(2/pi) * (x + 0.044715 x^3)))
+ */
 double oracle_activation(double x, int act)
 {
     if (act == ORACLE_ACT_RELU)
         return x > 0.0 ? x : 0.0;
     if (act == ORACLE_ACT_GELU)
         return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));
+    if (act == ORACLE_ACT_SILU)
+        return x / (1.0 + exp(-x));
+    if (act == ORACLE_ACT_GELU_TANH) {
+        const double pi = 3.14159265358979323846;
+        return 0.5 * x * (1.0 + tanh(sqrt(2.0 / pi) * (x + 0.044715 * x * x * x)));
+    }
     return x;
 }
 

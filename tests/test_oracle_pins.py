@@ -548,3 +548,106 @@ def test_fused_residual_in_fp32():
     got = oracle.gemm_fused(A, B, act="gelu", residual=R, threads=1)
     assert np.array_equal(got, base + R.astype(np.float64))
     assert not np.array_equal(got, base + dec(R.astype(np.float16)))
+
+
+# ----------------------------------------------------------------------------- SiLU and the tanh form of GELU
+# Standard definitions (the adoption page names activation fusion without formulas): SiLU is
+# x * sigmoid(x), checked against scipy's expit; the tanh form of GELU is checked against
+# torch's own implementation (gelu(approximate="tanh")) in float64.
+
+from scipy.special import expit  # noqa: E402
+
+
+def _points():
+    return f16(np.concatenate([np.linspace(-12, 12, 97), [-1.0, 1.0, 0.0, 1e-3, -1e-3, 30.0, -30.0]]))
+
+
+def _act_row(g, act):
+    xb = _points()
+    return dec(xb), g(np.ones((1, 1), np.float16), xb.reshape(1, -1), None, act, None)[0]
+
+
+def apin_silu_library(g):
+    x, out = _act_row(g, "silu")
+    assert np.all(np.abs(out - x * expit(x)) <= 4e-16 * (1 + np.abs(x))), np.max(np.abs(out - x * expit(x)))
+
+
+def apin_gelu_tanh_library(g):
+    import torch
+    x, out = _act_row(g, "gelu_tanh")
+    want = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    assert np.all(np.abs(out - want) <= 1e-15 * (1 + np.abs(x))), np.max(np.abs(out - want))
+
+
+def apin_sigmoid_forms_limits(g):
+    for act in ("silu", "gelu_tanh"):
+        x, out = _act_row(g, act)
+        assert out[np.argmin(np.abs(x))] == 0.0                      # act(0) = 0
+        big = x >= 12
+        assert np.all(np.abs(out[big] - x[big]) <= 1e-4 * x[big])     # act(x) -> x
+        assert np.all(np.abs(out[x <= -12]) <= 1e-4)                  # act(x) -> 0
+    # SiLU(x) - SiLU(-x) = x, and the tanh-GELU obeys the same symmetry
+    xb = f16(np.linspace(0, 6, 25))
+    for act in ("silu", "gelu_tanh"):
+        pos = g(np.ones((1, 1), np.float16), xb.reshape(1, -1), None, act, None)[0]
+        neg = g(-np.ones((1, 1), np.float16), xb.reshape(1, -1), None, act, None)[0]
+        assert np.all(np.abs((pos - neg) - dec(xb)) <= 1e-14 * (1 + dec(xb))), act
+
+
+APINS = [apin_silu_library, apin_gelu_tanh_library, apin_sigmoid_forms_limits]
+
+
+@pytest.mark.parametrize("pin", APINS, ids=lambda p: p.__name__)
+def test_oracle_activation_pins(pin):
+    pin(oracle_fused)
+
+
+def _aref(A, B, bias, act, R):
+    import torch
+    C = dec(A) @ dec(B)
+    if bias is not None:
+        C = C + dec(bias)[None, :]
+    if act == "silu":
+        C = C * expit(C)
+    elif act == "gelu_tanh":
+        C = torch.nn.functional.gelu(torch.from_numpy(C), approximate="tanh").numpy()
+    elif act == "gelu":
+        C = _gelu_scipy(C)
+    elif act == "relu":
+        C = np.maximum(C, 0.0)
+    return C + (dec(R) if R is not None else 0.0)
+
+
+def amutant_silu_sign(A, B, bias, act, R):
+    if act == "silu":
+        C = dec(A) @ dec(B) + (dec(bias)[None, :] if bias is not None else 0.0)
+        return C * expit(-C)
+    return _aref(A, B, bias, act, R)
+
+
+def amutant_gelu_tanh_without_cubic(A, B, bias, act, R):
+    if act == "gelu_tanh":
+        C = dec(A) @ dec(B) + (dec(bias)[None, :] if bias is not None else 0.0)
+        return 0.5 * C * (1 + np.tanh(math.sqrt(2 / math.pi) * C))
+    return _aref(A, B, bias, act, R)
+
+
+def amutant_silu_is_exact_gelu(A, B, bias, act, R):
+    return _aref(A, B, bias, "gelu" if act == "silu" else act, R)
+
+
+def test_activation_numpy_copy_passes_pins():
+    for pin in APINS:
+        pin(_aref)
+
+
+@pytest.mark.parametrize("mutant", [amutant_silu_sign, amutant_gelu_tanh_without_cubic, amutant_silu_is_exact_gelu],
+                         ids=lambda m: m.__name__)
+def test_activation_planted_mistake_is_caught(mutant):
+    failed = []
+    for pin in APINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"{mutant.__name__} passed every pin"
