@@ -253,8 +253,10 @@ tlg_status tlg_gemm_op(int64_t M, int64_t N, int64_t K,
 /* Activations of the fused epilogue. */
 typedef enum tlg_activation {
     TLG_ACT_NONE = 0,
-    TLG_ACT_RELU = 1, /* max(x, 0) */
-    TLG_ACT_GELU = 2  /* x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)), the exact (erf) form */
+    TLG_ACT_RELU = 1,      /* max(x, 0) */
+    TLG_ACT_GELU = 2,      /* x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)), the exact (erf) form */
+    TLG_ACT_SILU = 3,      /* x * sigmoid(x) = x / (1 + exp(-x)) */
+    TLG_ACT_GELU_TANH = 4  /* x/2 * (1 + tanh(sqrt(2/pi) * (x + 0.044715 x^3))) */
 } tlg_activation;
 
 /*
@@ -275,7 +277,7 @@ typedef enum tlg_activation {
  * names fusing an activation and a residual connection into the GEMM;
  * section 4.2 gives the bias-by-column-then-ReLU form (bias, TLG_ACT_RELU,
  * no residual, fp16 C is exactly tlg_gemm_bias_relu_f16).  The pages print
- * no GELU formula; the exact erf form is used.
+ * no activation formulas; each activation is its standard definition.
  */
 typedef struct tlg_fused_epilogue {
     const void *bias;

@@ -107,7 +107,7 @@ def test_fused_epilogue_host_side_rejections(lib_path):
                                   c, ldc, out, None, None, 0, None)
 
     E = tlg.tlg_fused_epilogue
-    assert call(E(None, 3, None, 0)) == tlg.TLG_ERR_INVALID_ARG          # no such activation
+    assert call(E(None, 5, None, 0)) == tlg.TLG_ERR_INVALID_ARG          # no such activation
     assert call(E(None, -1, None, 0)) == tlg.TLG_ERR_INVALID_ARG
     assert call(E(None, 2, C + 64, 8)) == tlg.TLG_ERR_INVALID_ARG        # residual overlaps C, shifted
     assert call(E(None, 2, C, 16)) == tlg.TLG_ERR_INVALID_ARG            # same base, other stride

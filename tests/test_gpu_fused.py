@@ -24,7 +24,7 @@ from gpu_util import Padded
 pytestmark = pytest.mark.gpu
 
 TILES = [(1, 64, 8), (1, 128, 6), (1, 256, 4), (2, 128, 8), (2, 256, 6), (2, 512, 4)]
-ACTS = ["none", "relu", "gelu"]
+ACTS = ["none", "relu", "gelu", "silu", "gelu_tanh"]
 
 
 @pytest.fixture(scope="module")
@@ -59,7 +59,7 @@ def run_fused(tlg, A, B, bias, act, R, out, cfg=None, op_a="N", op_b="N", extra=
         pr = Padded(R, M, N, cdt, al[3], extra[3])
     db = bias.cuda() if bias is not None else None
     epi = tlg.tlg_fused_epilogue(db.data_ptr() if db is not None else None,
-                                 {"none": 0, "relu": 1, "gelu": 2}[act], None, 0)
+                                 {"none": 0, "relu": 1, "gelu": 2, "silu": 3, "gelu_tanh": 4}[act], None, 0)
     if inplace:
         epi.residual, epi.ldr = pc.ptr(), pc.ld
     elif pr is not None:
@@ -258,3 +258,17 @@ def test_argument_errors_on_device(tlg):
         tlg.tlg_gemm_fused(A, A, activation="tanh")
     rc, code = tlg.tlg_device_error(clear=True)
     assert rc == 0 and code == 0
+
+
+@pytest.mark.parametrize("act", ["silu", "gelu_tanh"])
+def test_sigmoid_form_activations_pointwise(tlg, act):
+    # A = I: C = act(B) at fp16 points in [-12, 12]; fp32 results within a few fp32 ulp-scale
+    # errors of the fp64 definitions
+    N = 1024
+    x = torch.linspace(-12, 12, 64 * N).reshape(64, N).half()
+    A = torch.eye(64, dtype=torch.float16)
+    got = tlg.tlg_gemm_fused(A.cuda(), x.cuda(), activation=act, out="f32")
+    torch.cuda.synchronize()
+    ref = oracle.gemm_fused(A, x, act=act)
+    err = np.abs(got.double().cpu().numpy() - ref)
+    assert err.max() <= 2e-6 * (1 + np.abs(ref).max()), err.max()

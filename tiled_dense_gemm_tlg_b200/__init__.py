@@ -43,8 +43,9 @@ TLG_OK, TLG_ERR_INVALID_ARG, TLG_ERR_ALIGNMENT, TLG_ERR_UNSUPPORTED, TLG_ERR_CUD
 TLG_OUT_F32, TLG_OUT_F16 = 0, 1
 TLG_EPI_NONE, TLG_EPI_BIAS_RELU = 0, 1
 TLG_OP_N, TLG_OP_T = 0, 1
-TLG_ACT_NONE, TLG_ACT_RELU, TLG_ACT_GELU = 0, 1, 2
-_ACT = {"none": TLG_ACT_NONE, "relu": TLG_ACT_RELU, "gelu": TLG_ACT_GELU}
+TLG_ACT_NONE, TLG_ACT_RELU, TLG_ACT_GELU, TLG_ACT_SILU, TLG_ACT_GELU_TANH = 0, 1, 2, 3, 4
+_ACT = {"none": TLG_ACT_NONE, "relu": TLG_ACT_RELU, "gelu": TLG_ACT_GELU, "silu": TLG_ACT_SILU,
+        "gelu_tanh": TLG_ACT_GELU_TANH}
 
 EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
             "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_gemm_workspace_size_op", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
@@ -248,7 +249,7 @@ def tlg_gemm_fused(A: torch.Tensor, B: torch.Tensor, op_a: str = "N", op_b: str 
                    workspace: torch.Tensor | None = None, stream=None):
     """C = act(op(A).op(B) + bias[col]) + residual[row, col].
 
-    ``activation``: "none", "relu" or "gelu" (exact erf form).  ``residual``:
+    ``activation``: "none", "relu", "gelu" (exact erf form), "silu" or "gelu_tanh".  ``residual``:
     an M x N row-major tensor of C's type (fp16 for out="f16", fp32 for
     out="f32"); it may be ``C`` itself for an in-place residual connection.
     Operands and ``op_a`` / ``op_b`` as ``tlg_gemm_op``."""

@@ -268,7 +268,8 @@ bool encode_2d(CUtensorMap *tm, CUtensorMapDataType dtype, const void *base, uin
   return r == CUDA_SUCCESS;
 }
 
-static_assert(kActNone == TLG_ACT_NONE && kActRelu == TLG_ACT_RELU && kActGelu == TLG_ACT_GELU,
+static_assert(kActNone == TLG_ACT_NONE && kActRelu == TLG_ACT_RELU && kActGelu == TLG_ACT_GELU &&
+                  kActSilu == TLG_ACT_SILU && kActGeluTanh == TLG_ACT_GELU_TANH,
               "the kernels' activation codes are tlg_activation's values");
 
 // The epilogue of one call, from either interface: bias, activation and
@@ -302,7 +303,8 @@ tlg_status fused_epilogue(tlg_out out, const tlg_fused_epilogue *d, Epi *e) {
   *e = Epi{};
   if (d == nullptr) return TLG_OK;
   if (d->activation != TLG_ACT_NONE && d->activation != TLG_ACT_RELU &&
-      d->activation != TLG_ACT_GELU)
+      d->activation != TLG_ACT_GELU && d->activation != TLG_ACT_SILU &&
+      d->activation != TLG_ACT_GELU_TANH)
     return TLG_ERR_INVALID_ARG;
   e->bias = d->bias;
   e->act = d->activation;

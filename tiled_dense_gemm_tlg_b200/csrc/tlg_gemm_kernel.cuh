@@ -169,6 +169,8 @@ constexpr int kEpiBiasRelu = 2;
 constexpr int kActNone = 0;
 constexpr int kActRelu = 1;
 constexpr int kActGelu = 2;
+constexpr int kActSilu = 3;
+constexpr int kActGeluTanh = 4;
 
 // Hardware approximations (PTX rcp.approx / ex2.approx, flushing subnormals).
 __device__ __forceinline__ float rcp_approx(float x) {
@@ -206,9 +208,32 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return x * (x < 0.0f ? q : 1.0f - q);
 }
 
+// SiLU and the tanh form of GELU are both x * sigmoid(c1 x + c3 x^3):
+//   SiLU:      c1 = 1,                 c3 = 0;
+//   tanh GELU: x/2 (1 + tanh(y)) = x sigmoid(2y) with y = sqrt(2/pi) (x + 0.044715 x^3),
+//              so c1 = 2 sqrt(2/pi),  c3 = 0.044715 c1.
+// sigmoid(z) = 1 / (1 + 2^(-z log2 e)); one code path for both, with the
+// coefficients chosen per call.
+struct SigmoidForm {
+  float c1, c3;  // already multiplied by -log2(e)
+};
+
+__device__ __forceinline__ SigmoidForm sigmoid_form(int act) {
+  constexpr float kNegLog2e = -1.4426950408889634f;
+  constexpr float kTanhC1 = 1.5957691216057308f;  // 2 sqrt(2/pi)
+  if (act == kActSilu) return {kNegLog2e, 0.0f};
+  return {kNegLog2e * kTanhC1, kNegLog2e * kTanhC1 * 0.044715f};
+}
+
+__device__ __forceinline__ float sigmoid_form_apply(SigmoidForm f, float x) {
+  const float z = x * fmaf(f.c3, x * x, f.c1);  // -(c1 x + c3 x^3) log2(e)
+  return x * rcp_approx(1.0f + ex2_approx(z));
+}
+
 __device__ __forceinline__ float activate(int act, float x) {
   if (act == kActRelu) return fmaxf(x, 0.0f);
   if (act == kActGelu) return gelu_erf(x);
+  if (act == kActSilu || act == kActGeluTanh) return sigmoid_form_apply(sigmoid_form(act), x);
   return x;
 }
 
@@ -221,6 +246,10 @@ __device__ __forceinline__ void activate_32(int act, float (&v)[32]) {
   } else if (act == kActGelu) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+  } else if (act == kActSilu || act == kActGeluTanh) {
+    const SigmoidForm f = sigmoid_form(act);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = sigmoid_form_apply(f, v[j]);
   }
 }
 
