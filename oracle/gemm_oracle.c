@@ -18,9 +18,9 @@
  *     the ReLU: "domestic-GPU TileLang adoption" (xdnf.cn/news/333523)
  *     section 4.2; the same page's section 4.1 names fusing an activation
  *     and a residual connection into the GEMM, written here as
- *     ref = act(A.B + bias[j]) + R[i][j] with act = none, ReLU or GELU.
- *     GELU is the exact form x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)) (the
- *     pages give no formula; this is its standard definition).
+ *     ref = act(A.B + bias[j]) + R[i][j] with act = none, ReLU, GELU, SiLU
+ *     or GELU's tanh form.  The pages give no activation formulas; each is
+ *     its standard definition (oracle_activation below).
  *
  * The accumulation is fp64 (every fp16 x fp16 product is exact in fp64), so
  * the result is the exact sum up to fp64 rounding.  The k order is ascending
