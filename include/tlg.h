@@ -71,7 +71,7 @@ extern "C" {
 typedef enum tlg_status {
     TLG_OK = 0,
     TLG_ERR_INVALID_ARG = 1, /* negative size, null/host pointer, ld too small, overlap */
-    TLG_ERR_ALIGNMENT = 2,   /* pointer or row stride breaks the 16-byte rule */
+    TLG_ERR_ALIGNMENT = 2,   /* pointer not aligned to its element; workspace not 256-byte aligned */
     TLG_ERR_UNSUPPORTED = 3, /* not an sm_100 device, size beyond 2^31-1, bad config */
     TLG_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
     TLG_ERR_TIMEOUT = 5      /* a kernel reported a pipeline wait past its time limit */

@@ -934,8 +934,8 @@ const char *tlg_status_string(tlg_status status) {
       return "TLG_ERR_INVALID_ARG: bad size, null or host pointer, ld too small, overlapping "
              "buffers, or a workspace too small for the requested split";
     case TLG_ERR_ALIGNMENT:
-      return "TLG_ERR_ALIGNMENT: pointers must be 16-byte aligned (the workspace 256-byte) and row "
-             "strides multiples of 16 bytes";
+      return "TLG_ERR_ALIGNMENT: a matrix or bias pointer not aligned to its element (2 bytes for "
+             "fp16, 4 for fp32), or a workspace not 256-byte aligned";
     case TLG_ERR_UNSUPPORTED:
       return "TLG_ERR_UNSUPPORTED: device is not sm_100, size too large, or configuration not "
              "provided";

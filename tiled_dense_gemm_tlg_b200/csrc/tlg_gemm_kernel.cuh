@@ -4,24 +4,34 @@
 // (row block, column block), an fp32 accumulator per tile, operand tiles of
 // A[rows, k-block] and B[k-block, cols] staged in shared memory by a
 // multi-stage pipeline over the K loop ("tilelang operator-compilation
-// walkthrough", lqnn.cn/news/222844, section 2.1) -- mapped onto Blackwell:
+// walkthrough", lqnn.cn/news/222844, section 2.1) -- mapped onto Blackwell.
+// A tile is 128*CG rows (CG = 1 CTA, or a 2-CTA cluster issuing
+// tcgen05.mma.cta_group::2) by BN*NH columns (NH = 2: two MMA halves that fill
+// TMEM):
 //
 //   warp 0 (one lane)  producer: TMA loads of the A and B tiles of each
 //                      k-block into a STAGES-deep ring, one mbarrier pair per
 //                      slot (full: bytes landed; empty: the MMAs read it).
-//   warp 1 (one lane)  MMA issuer: tcgen05.mma 128 x BN x 16 into a TMEM
-//                      accumulator; two accumulators alternate so the
-//                      epilogue of tile i overlaps the main loop of tile i+1.
-//                      Warp 1 also owns the TMEM allocation.
-//   warps 2-5          epilogue: tcgen05.ld of the accumulator, then bias,
-//                      ReLU and the output cast ("domestic-GPU TileLang
-//                      adoption", xdnf.cn/news/333523, section 4.2), staged in
-//                      shared memory and written by TMA bulk-tensor stores,
-//                      which clip the rows and columns outside M x N.
+//   warp 1 (one lane)  MMA issuer (the pair's leader CTA): tcgen05.mma into a
+//                      TMEM accumulator; with NH == 1 two accumulators
+//                      alternate, so the epilogue of tile i overlaps the main
+//                      loop of tile i+1.  Warp 1 also owns the TMEM allocation.
+//   warps 2-5          epilogue: tcgen05.ld of the accumulator, the fused
+//                      epilogue of the build (none; bias + ReLU, "domestic-GPU
+//                      TileLang adoption", xdnf.cn/news/333523, section 4.2;
+//                      or bias, activation and residual chosen per call,
+//                      section 4.1) and the output cast, staged in shared
+//                      memory and written by TMA bulk-tensor stores, which clip
+//                      the rows and columns outside M x N.
+//   warps 6-9          plain-load builds only: loader warps that fill the ring
+//                      with ordinary loads for operands TMA cannot describe
+//                      (warp 0 then idles).
 //
-// CTAs are persistent (one per SM) and walk the tile list with a stride of
-// gridDim.x; consecutive tiles are grouped by `raster_group` row blocks so
-// the CTAs of one wave share A and B tiles in L2.
+// Work units (CTAs, or CTA pairs) are persistent and walk the tile list with a
+// stride of the unit count; consecutive tiles are grouped by `raster_group`
+// row blocks so the units of one wave share A and B tiles in L2.  An optional
+// split-K tail cuts the tiles left after the last whole wave into k-slices
+// whose fp32 partials the last-arriving slice sums in a fixed order.
 //
 // Ragged M, N and K need no special code in the main loop: the TMA unit fills
 // out-of-range elements of a box with zeros, so the last k-block adds 0 for
