@@ -232,7 +232,8 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
       Schedule sch;
       if (!plan(tiles, resident, num_kb, split, k.cta_group, k.block_n, &sch)) continue;
       if (r.split_k == 0 && split > 1 && (sch.dp_tiles == 0 || sch.workspace > ws_bytes)) continue;
-      const double per_unit_tiles = static_cast<double>(tiles + sch.units - 1) / sch.units;
+      // the busiest unit's tile count, each tile paying the exposed part of its epilogue
+      const double per_unit_tiles = static_cast<double>((tiles + sch.units - 1) / sch.units);
       const double cost = (sch.cost + per_unit_tiles * k.exposed_kb) *
                           static_cast<double>(tile_m * k.block_n) / (k.cta_group * k.eff);
       if (!found || cost < best_cost * 0.999) {
