@@ -123,3 +123,42 @@ def test_size_query_for_aligned_operands_is_the_split_scratch(tlg):
     Ao = torch.empty((M, K + 1), dtype=torch.float16, device="cuda")[:, :K]
     more = tlg.tlg_gemm_workspace_size_op(Ao, B, C)
     assert more >= tlg.tlg_gemm_workspace_size(M, N, K, "f16", False) + M * K * 2
+
+
+def test_size_query_bytes_hold_the_split_and_the_copy(tlg):
+    # 108 pair tiles (3072 x 2304): one whole wave, then a tail the automatic choice cuts in two
+    # along K when the workspace holds the slices' partial sums.  Only A needs a copy.  With
+    # exactly the size query's bytes the call must take the same schedule as the query: the
+    # split scratch first, then A's aligned copy, ending at the workspace's last byte.
+    M, N, K = 3072, 2304, 512
+    A, B, bias = wl.make_operands(M, N, K, "uniform", bias=True, seed=406)
+    lib = tlg.raw_library()
+    ra = Raw(A, M, K, K + 1, torch.float16, 0)
+    Bd, C = B.cuda(), torch.empty((M, N), dtype=torch.float16, device="cuda")
+    full = ctypes.c_size_t(0)
+    rcq = lib.tlg_gemm_workspace_size_op(M, N, K, 0, ra.ptr(), ra.ld, 0, Bd.data_ptr(), N, C.data_ptr(), N,
+                                         tlg.TLG_OUT_F16, None, ctypes.byref(full))
+    assert rcq == 0, tlg.tlg_status_string(rcq)
+    a_copy = M * K * 2  # rows of 1024 bytes: already 16- and 256-byte multiples
+    split_ws = tlg.tlg_gemm_workspace_size(M, N, K, "f16", True)
+    assert split_ws > 4096, "the automatic choice no longer splits this shape"
+    assert full.value == (split_ws + 255) // 256 * 256 + a_copy
+    ws = tlg.tlg_workspace(full.value)
+    ws[4096:] = 0xFF
+    dbias = bias.cuda()
+    epi = tlg.tlg_fused_epilogue(dbias.data_ptr(), 1, None, 0)
+    rc = lib.tlg_gemm_fused(M, N, K, 0, ra.ptr(), ra.ld, 0, Bd.data_ptr(), N, ctypes.byref(epi), C.data_ptr(), N,
+                            tlg.TLG_OUT_F16, None, ws.data_ptr(), full.value,
+                            int(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, tlg.tlg_status_string(rc)
+    torch.cuda.synchronize()
+    assert ra.guard_ok()
+    assert int(ws[:4096].count_nonzero()) == 0, "split-K counters left non-zero"
+    tail = ws[full.value - a_copy:].view(torch.float16).view(M, K).cpu()
+    assert torch.equal(tail.view(torch.int16), A.view(torch.int16)), "A's copy is not where the query put it"
+    assert int((ws[4096:4096 + 1024] != 0xFF).sum()) > 0, "no partial sums: the split tail was not taken"
+    rows = np.arange(0, M, 97)
+    got = C[torch.from_numpy(rows).cuda()].double().cpu().numpy()
+    ref = oracle.gemm(A[torch.from_numpy(rows)], B, bias=bias, relu=True)
+    ok, worst, idx = oracle.within_tolerance(got, ref, "f16")
+    assert ok, (worst, idx)

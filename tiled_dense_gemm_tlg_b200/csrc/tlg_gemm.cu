@@ -570,9 +570,11 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   tlg_status rs = TLG_ERR_UNSUPPORTED;
   size_t copy_base = 0;
   if ((cp.a || cp.b) && ws_bytes >= kCounterBytes + cp.ab_bytes()) {
-    // the TMA path with copies of A and/or B, split scratch from what is left
-    rs = resolve(dev, info.sm_count, M, N, K, f16, ek, at, bt, false, req,
-                 ws_bytes - kCounterBytes - cp.ab_bytes(), &rv);
+    // The TMA path with copies of A and/or B.  The split scratch (counters
+    // included) starts the workspace and the copies follow it, 256-byte
+    // aligned, so the scratch may take what the copies leave, rounded down.
+    const size_t split_room = (ws_bytes - cp.ab_bytes()) / kCopyAlign * kCopyAlign;
+    rs = resolve(dev, info.sm_count, M, N, K, f16, ek, at, bt, false, req, split_room, &rv);
     if (rs == TLG_OK) {
       copy_ab = true;
       copy_base = round_up_sz(std::max<size_t>(rv.sched.workspace, kCounterBytes), kCopyAlign);
