@@ -442,12 +442,12 @@ def main(argv=None):
         """The library's rule for a TMA operand: 16-byte base and row stride."""
         return x.data_ptr() % 16 == 0 and (x.stride(0) * x.element_size()) % 16 == 0
 
-    # Kernels one call launches: the GEMM, plus an aligned copy of each matrix TMA cannot
-    # describe when the workspace holds the copies (it does: its size comes from the size
-    # query that counts them).
+    # Kernels one call launches: the GEMM, plus one kernel copying whichever of A and B TMA
+    # cannot describe and one copying such a C out, when the workspace holds the copies (it
+    # does: its size comes from the size query that counts them).
     copies = 0
     if ws_bytes > 0 and (args.ld_pad or at or bt):
-        copies = sum(not tma_describable(x) for x in (dA, dB, dC))
+        copies = int(not (tma_describable(dA) and tma_describable(dB))) + int(not tma_describable(dC))
     launches_per_step = 1 + copies
     use_ex = (ws is not None or override is not None) and not use_op and not fused
     entry = "tlg_gemm_op" if use_op else ("tlg_gemm_ex" if use_ex else plain_name)
@@ -643,7 +643,7 @@ def main(argv=None):
     if copies:
         # The step's events bracket the GEMM and its copies: the figure is the whole call's, and
         # the stored per-kernel DRAM traffic does not describe it.
-        roofline["covers"] = f"the whole call: the GEMM and {copies} aligned copies, one launch each"
+        roofline["covers"] = f"the whole call: the GEMM and {copies} aligned-copy kernel(s)"
         roofline["traffic"] = None
 
     cpu = None

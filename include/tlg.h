@@ -326,7 +326,11 @@ tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
  * layout in the workspace first and runs the TMA path on the copies; such a
  * C is produced in the workspace and copied out at the end.  Each copy moves
  * every byte once, so a call with odd strides then runs near the speed of
- * an aligned one instead of on the plain-load path.  With less workspace the
+ * an aligned one instead of on the plain-load path.  Such a call enqueues up
+ * to three kernels: one copying A and B, the GEMM, and the copy of C; the
+ * GEMM and the copy of C start as programmatic dependents of the kernel
+ * before them (their set-up overlaps its end; each waits for it before
+ * touching memory).  With less workspace the
  * call still succeeds on the plain-load path (A and B copies are made only
  * when both fit; a C copy when it fits after them).  The copies never touch
  * the workspace's first 4 KB (the split-K counters).  0 when every matrix is

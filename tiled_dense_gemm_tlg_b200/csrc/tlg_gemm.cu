@@ -420,17 +420,38 @@ struct PieceIter {
   }
 };
 
+// One matrix of a copy: `rows` rows of `row_bytes` bytes, strides in bytes.
+struct CopyJob {
+  const char *src;
+  int64_t src_ld;
+  char *dst;
+  int64_t dst_ld;
+  int64_t rows;
+  int64_t row_bytes;
+};
+
 // Into the workspace: dst (16-byte base and row stride) <- src (any address).
 // Row r's output block b is src bytes [16b, 16b + 16) of the row, which sit in
 // the aligned source blocks b and b + 1 counted from the row's first byte
 // rounded down to 16.  The last output block of a row may run past row_bytes
 // into the row's padding (the layout rounds rows up to 16 bytes).
+// One launch copies A and B: blocks [0, j1_first) take j0, the rest j1.  The
+// GEMM that reads the copies may be launched as a programmatic dependent: it
+// is let in at once and waits for this grid before it touches global memory.
 __global__ void __launch_bounds__(kCopyThreads, kCopyBlocksPerSm)
-    copy_in_kernel(const char *__restrict__ src, int64_t src_ld_bytes, char *__restrict__ dst,
-                   int64_t dst_ld_bytes, int64_t rows, int64_t row_bytes) {
+    copy_in_kernel(CopyJob j0, CopyJob j1, unsigned j1_first) {
+  grid_launch_dependents();
+  const bool second = blockIdx.x >= j1_first;
+  const char *const src = second ? j1.src : j0.src;
+  char *const dst = second ? j1.dst : j0.dst;
+  const int64_t src_ld_bytes = second ? j1.src_ld : j0.src_ld;
+  const int64_t dst_ld_bytes = second ? j1.dst_ld : j0.dst_ld;
+  const int64_t rows = second ? j1.rows : j0.rows;
+  const int64_t row_bytes = second ? j1.row_bytes : j0.row_bytes;
+  const unsigned block = second ? blockIdx.x - j1_first : blockIdx.x;
   const int lane = threadIdx.x & 31;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kCopyWarps;
-  PieceIter it(static_cast<int64_t>(blockIdx.x) * kCopyWarps + (threadIdx.x >> 5), nwarps,
+  const int64_t nwarps = static_cast<int64_t>(second ? gridDim.x - j1_first : j1_first) * kCopyWarps;
+  PieceIter it(static_cast<int64_t>(block) * kCopyWarps + (threadIdx.x >> 5), nwarps,
                (row_bytes + 511) / 512);
   while (it.r < rows) {
     uint4 lo[kCopyUnroll], next[kCopyUnroll];
@@ -472,10 +493,16 @@ __global__ void __launch_bounds__(kCopyThreads, kCopyBlocksPerSm)
 // [16b - t, 16b - t + 16), t the row's offset in its first block, which are
 // bytes [16 - t, 32 - t) of source blocks b - 1 and b.  Blocks wholly inside
 // the row are stored whole; the row's first and last blocks element by element.
+// Launched as a programmatic dependent of the GEMM that writes src: it waits
+// for that grid before touching global memory.
 template <int ESZ>
 __global__ void __launch_bounds__(kCopyThreads, kCopyBlocksPerSm)
-    copy_out_kernel(const char *__restrict__ src, int64_t src_ld_bytes, char *__restrict__ dst,
-                    int64_t dst_ld_bytes, int64_t rows, int64_t row_bytes) {
+    copy_out_kernel(CopyJob j) {
+  grid_dependency_wait();
+  const char *const src = j.src;
+  char *const dst = j.dst;
+  const int64_t src_ld_bytes = j.src_ld, dst_ld_bytes = j.dst_ld;
+  const int64_t rows = j.rows, row_bytes = j.row_bytes;
   const int lane = threadIdx.x & 31;
   const int64_t src_blocks = (row_bytes + 15) / 16;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kCopyWarps;
@@ -536,29 +563,54 @@ int64_t aligned_ld(int64_t cols, int64_t esz) {
   return static_cast<int64_t>(round_up_sz(static_cast<size_t>(cols * esz), 16)) / esz;
 }
 
-// dst <- src, rows x cols elements of esz bytes, row strides in elements.
-// One of the two must be 16-byte aligned in base and row stride (the
-// workspace side); the other needs only element alignment.
-tlg_status launch_copy(const void *src, int64_t src_ld, void *dst, int64_t dst_ld, int64_t rows,
-                       int64_t cols, int64_t esz, int sms, cudaStream_t s) {
-  auto aligned = [esz](const void *q, int64_t ld) { return aligned16(q) && (ld * esz) % 16 == 0; };
-  const int64_t row_bytes = cols * esz;
-  const int64_t per_row = aligned(dst, dst_ld) ? (row_bytes + 511) / 512 : ((row_bytes + 29) / 16 + 31) / 32;
-  const int64_t warps = rows * per_row;
+bool aligned_rows(const void *q, int64_t ld_bytes) { return aligned16(q) && ld_bytes % 16 == 0; }
+
+// Blocks for `items` warp-sized pieces, at most `cap`.
+int64_t copy_blocks(int64_t items, int64_t cap) {
+  return std::max<int64_t>(1, std::min<int64_t>(cap, (items + kCopyWarps - 1) / kCopyWarps));
+}
+
+// Copies of A and/or B into the workspace (dst rows 16-byte aligned), one
+// launch; b may be null.  The blocks (one wave at most) are shared in
+// proportion to the two matrices' sizes.
+tlg_status launch_copy_in(const CopyJob &a, const CopyJob *b, int sms, cudaStream_t s) {
+  // the workspace side must be 16-byte aligned (never otherwise: it is planned so)
+  if (!aligned_rows(a.dst, a.dst_ld) || (b != nullptr && !aligned_rows(b->dst, b->dst_ld)))
+    return TLG_ERR_INVALID_ARG;
   const int64_t cap = static_cast<int64_t>(std::max(sms, 1)) * kCopyBlocksPerSm;
-  const unsigned blocks =
-      static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(cap, (warps + kCopyWarps - 1) / kCopyWarps)));
-  const char *sp = static_cast<const char *>(src);
-  char *dp = static_cast<char *>(dst);
-  if (aligned(dst, dst_ld))
-    copy_in_kernel<<<blocks, kCopyThreads, 0, s>>>(sp, src_ld * esz, dp, dst_ld * esz, rows, row_bytes);
-  else if (!aligned(src, src_ld))
-    return TLG_ERR_INVALID_ARG;  // never planned: one side is always the workspace
-  else if (esz == 4)
-    copy_out_kernel<4><<<blocks, kCopyThreads, 0, s>>>(sp, src_ld * esz, dp, dst_ld * esz, rows, row_bytes);
-  else
-    copy_out_kernel<2><<<blocks, kCopyThreads, 0, s>>>(sp, src_ld * esz, dp, dst_ld * esz, rows, row_bytes);
+  const int64_t ia = a.rows * ((a.row_bytes + 511) / 512);
+  const int64_t ib = b != nullptr ? b->rows * ((b->row_bytes + 511) / 512) : 0;
+  int64_t na = copy_blocks(ia, cap), nb = b != nullptr ? copy_blocks(ib, cap) : 0;
+  if (b != nullptr && na + nb > cap) {
+    na = std::max<int64_t>(1, std::min<int64_t>(na, (cap * ia) / (ia + ib)));
+    nb = std::max<int64_t>(1, std::min<int64_t>(nb, cap - na));
+  }
+  copy_in_kernel<<<static_cast<unsigned>(na + nb), kCopyThreads, 0, s>>>(a, b != nullptr ? *b : a,
+                                                                        static_cast<unsigned>(na));
   if (cudaPeekAtLastError() != cudaSuccess) {
+    cudaGetLastError();
+    return TLG_ERR_CUDA;
+  }
+  return TLG_OK;
+}
+
+// The copy of C out of the workspace (src rows 16-byte aligned), launched as
+// a programmatic dependent of the GEMM before it.
+tlg_status launch_copy_out(const CopyJob &c, int64_t esz, int sms, cudaStream_t s) {
+  if (!aligned_rows(c.src, c.src_ld)) return TLG_ERR_INVALID_ARG;  // the workspace side, as planned
+  const int64_t cap = static_cast<int64_t>(std::max(sms, 1)) * kCopyBlocksPerSm;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(copy_blocks(c.rows * (((c.row_bytes + 29) / 16 + 31) / 32), cap)));
+  cfg.blockDim = dim3(kCopyThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = esz == 4 ? cudaLaunchKernelEx(&cfg, copy_out_kernel<4>, c)
+                                 : cudaLaunchKernelEx(&cfg, copy_out_kernel<2>, c);
+  if (e != cudaSuccess) {
     cudaGetLastError();
     return TLG_ERR_CUDA;
   }
@@ -750,21 +802,23 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   int64_t lda_use = lda, ldb_use = ldb;
   if (copy_ab) {
     size_t off = copy_base;
+    CopyJob jobs[2];
+    int n = 0;
     if (cp.a) {
       const int64_t rows = at ? K : M, cols = at ? M : K;
       lda_use = aligned_ld(cols, 2);
-      const tlg_status cs = launch_copy(A, lda, wsb + off, lda_use, rows, cols, 2, info.sm_count, s);
-      if (cs != TLG_OK) return cs;
+      jobs[n++] = {static_cast<const char *>(A), lda * 2, wsb + off, lda_use * 2, rows, cols * 2};
       A_use = wsb + off;
       off += cp.a_bytes;
     }
     if (cp.b) {
       const int64_t rows = bt ? N : K, cols = bt ? K : N;
       ldb_use = aligned_ld(cols, 2);
-      const tlg_status cs = launch_copy(B, ldb, wsb + off, ldb_use, rows, cols, 2, info.sm_count, s);
-      if (cs != TLG_OK) return cs;
+      jobs[n++] = {static_cast<const char *>(B), ldb * 2, wsb + off, ldb_use * 2, rows, cols * 2};
       B_use = wsb + off;
     }
+    const tlg_status cs = launch_copy_in(jobs[0], n > 1 ? &jobs[1] : nullptr, info.sm_count, s);
+    if (cs != TLG_OK) return cs;
   }
   void *C_use = copy_c ? static_cast<void *>(wsb + c_off) : C;
   const int64_t ldc_use = copy_c ? aligned_ld(N, osz) : ldc;
@@ -816,10 +870,14 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   p.R = e.R;
   p.ldr = e.ldr;
   p.r_vec = (e.R != nullptr && aligned16(e.R) && (e.ldr * osz) % 16 == 0) ? 1 : 0;
+  // After this call's own copy kernel the GEMM starts as its programmatic
+  // dependent: its set-up overlaps the copy's tail.
   const tlg_status ls = fns_for(rv.idx, f16, ek, at, bt, plain)
-                             .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0, s);
+                             .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0 || copy_ab, s);
   if (ls != TLG_OK || !copy_c) return ls;
-  return launch_copy(C_use, aligned_ld(N, osz), C, ldc, M, N, osz, info.sm_count, s);
+  const CopyJob jc = {static_cast<const char *>(C_use), aligned_ld(N, osz) * osz, static_cast<char *>(C),
+                      ldc * osz, M, N * osz};
+  return launch_copy_out(jc, osz, info.sm_count, s);
 }
 
 // ---------------------------------------------------------------- allocation-free scratch
