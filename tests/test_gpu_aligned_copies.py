@@ -162,3 +162,41 @@ def test_size_query_bytes_hold_the_split_and_the_copy(tlg):
     ref = oracle.gemm(A[torch.from_numpy(rows)], B, bias=bias, relu=True)
     ok, worst, idx = oracle.within_tolerance(got, ref, "f16")
     assert ok, (worst, idx)
+
+
+def test_copy_chain_back_to_back(tlg):
+    # Calls whose A, B and C all need copies, issued back to back on one stream with two input
+    # sets alternating: the copy of A and B, the GEMM (a programmatic dependent of it) and the
+    # copy of C (a dependent of the GEMM) must each see the kernel before it complete.  A result
+    # that mixed in the other set's data would differ from that set's first result, which the
+    # oracle checks; the kernels are deterministic, so every repeat must match it bit for bit.
+    lib = tlg.raw_library()
+    M, N, K = 520, 264, 1000
+    sets = [wl.make_operands(M, N, K, "uniform", bias=True, seed=407 + i) for i in range(2)]
+    raws = []
+    for A, B, bias in sets:
+        ra = Raw(A, M, K, K + 1, torch.float16, 1)
+        rb = Raw(B, K, N, N + 3, torch.float16, 3)
+        raws.append((ra, rb, bias.cuda()))
+    rc_ = Raw(None, M, N, N + 1, torch.float16, 1)
+    full = ctypes.c_size_t(0)
+    ra0, rb0, _ = raws[0]
+    assert lib.tlg_gemm_workspace_size_op(M, N, K, 0, ra0.ptr(), ra0.ld, 0, rb0.ptr(), rb0.ld, rc_.ptr(), rc_.ld,
+                                          tlg.TLG_OUT_F16, None, ctypes.byref(full)) == 0
+    ws = tlg.tlg_workspace(full.value)
+    stream = int(torch.cuda.current_stream().cuda_stream)
+    outs = []
+    for it in range(12):
+        ra, rb, dbias = raws[it % 2]
+        rc = lib.tlg_gemm_op(M, N, K, 0, ra.ptr(), ra.ld, 0, rb.ptr(), rb.ld, dbias.data_ptr(), rc_.ptr(), rc_.ld,
+                             tlg.TLG_OUT_F16, tlg.TLG_EPI_BIAS_RELU, None, ws.data_ptr(), full.value, stream)
+        assert rc == 0, tlg.tlg_status_string(rc)
+        outs.append(rc_.matrix().clone())  # stream-ordered copy of this call's C
+    torch.cuda.synchronize()
+    assert rc_.guard_ok()
+    for i, (A, B, bias) in enumerate(sets):
+        got = outs[i].double().cpu().numpy()
+        ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B, bias=bias, relu=True), "f16")
+        assert ok, (i, worst, idx)
+    for it in range(2, 12):
+        assert torch.equal(outs[it].view(torch.int16), outs[it % 2].view(torch.int16)), it
