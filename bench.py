@@ -385,8 +385,9 @@ def main(argv=None):
     ap.add_argument("--layout", default="NN", choices=["NN", "NT", "TN", "TT"],
                     help="op(A), op(B): T = that operand is stored transposed (tlg_gemm_op)")
     ap.add_argument("--ld-pad", type=int, default=0,
-                    help="extra elements in every row stride (odd: strides TMA cannot describe, "
-                         "served by the plain-load path)")
+                    help="extra elements in every row stride (odd: strides TMA cannot describe; "
+                         "the bench passes the workspace the size query asks for, so the call "
+                         "copies such matrices into an aligned layout)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
