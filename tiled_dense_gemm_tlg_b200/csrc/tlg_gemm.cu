@@ -1,6 +1,7 @@
 // Host side of libtlg: argument checks, TMA descriptor encoding, the per-shape
 // configuration table, the work schedule and the launches behind the C
-// interface in tlg.h.
+// interface in tlg.h; also the small kernels around the GEMM (the K = 0 fill,
+// the aligned copies of operands TMA cannot describe, the timeout self-test).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
