@@ -200,3 +200,40 @@ def test_copy_chain_back_to_back(tlg):
         assert ok, (i, worst, idx)
     for it in range(2, 12):
         assert torch.equal(outs[it].view(torch.int16), outs[it % 2].view(torch.int16)), it
+
+
+@pytest.mark.parametrize("out", ["f16", "f32"])
+def test_large_copies_match_the_aligned_call_bit_for_bit(tlg, out):
+    # 4096 rows of 8 KB (fp16) or 16 KB (fp32): every warp of the copy kernels walks many row
+    # pieces.  The same GEMM configuration runs on aligned operands and on odd-stride ones
+    # (copied in, C copied out); the copies are exact, so the two Cs must agree bit for bit.
+    lib = tlg.raw_library()
+    M, N, K = 4096, 4096, 256
+    A, B, _ = wl.make_operands(M, N, K, "uniform", seed=408)
+    odt = torch.float32 if out == "f32" else torch.float16
+    o = tlg.TLG_OUT_F32 if out == "f32" else tlg.TLG_OUT_F16
+    cfg = tlg.tlg_config(cta_group=2, block_n=256, split_k=1)
+    stream = int(torch.cuda.current_stream().cuda_stream)
+    dA, dB = A.cuda(), B.cuda()
+    ref = torch.empty((M, N), dtype=odt, device="cuda")
+    rc = lib.tlg_gemm_op(M, N, K, 0, dA.data_ptr(), K, 0, dB.data_ptr(), N, None, ref.data_ptr(), N, o,
+                         tlg.TLG_EPI_NONE, ctypes.byref(cfg), None, 0, stream)
+    assert rc == 0, tlg.tlg_status_string(rc)
+    ra = Raw(A, M, K, K + 1, torch.float16, 1)
+    rb = Raw(B, K, N, N + 3, torch.float16, 5)
+    rc_ = Raw(None, M, N, N + 1, odt, 1)
+    full = ctypes.c_size_t(0)
+    assert lib.tlg_gemm_workspace_size_op(M, N, K, 0, ra.ptr(), ra.ld, 0, rb.ptr(), rb.ld, rc_.ptr(), rc_.ld, o,
+                                          ctypes.byref(cfg), ctypes.byref(full)) == 0
+    ws = tlg.tlg_workspace(full.value)
+    rc = lib.tlg_gemm_op(M, N, K, 0, ra.ptr(), ra.ld, 0, rb.ptr(), rb.ld, None, rc_.ptr(), rc_.ld, o,
+                         tlg.TLG_EPI_NONE, ctypes.byref(cfg), ws.data_ptr(), full.value, stream)
+    assert rc == 0, tlg.tlg_status_string(rc)
+    torch.cuda.synchronize()
+    assert all(r.guard_ok() for r in (ra, rb, rc_)), "guard band changed"
+    ityp = torch.int32 if out == "f32" else torch.int16
+    assert torch.equal(rc_.matrix().contiguous().view(ityp), ref.view(ityp))
+    rows = np.arange(0, M, 127)
+    got = ref[torch.from_numpy(rows).cuda()].double().cpu().numpy()
+    ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A[torch.from_numpy(rows)], B), out)
+    assert ok, (worst, idx)
