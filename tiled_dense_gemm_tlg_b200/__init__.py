@@ -48,8 +48,9 @@ _ACT = {"none": TLG_ACT_NONE, "relu": TLG_ACT_RELU, "gelu": TLG_ACT_GELU, "silu"
         "gelu_tanh": TLG_ACT_GELU_TANH}
 
 EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg_gemm_ex",
-            "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size", "tlg_gemm_workspace_size_op", "tlg_choose_config", "tlg_device_error", "tlg_selftest_timeout", "tlg_status_string",
-            "tlg_version")
+            "tlg_gemm_op", "tlg_gemm_fused", "tlg_gemm_ex_noalloc", "tlg_gemm_workspace_size",
+            "tlg_gemm_workspace_size_op", "tlg_choose_config", "tlg_device_error",
+            "tlg_selftest_timeout", "tlg_status_string", "tlg_version")
 
 
 class tlg_config(ctypes.Structure):
