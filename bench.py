@@ -26,6 +26,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -49,13 +50,21 @@ FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ("tlg_device.cuh", "tlg_gemm_kernel.cuh")  # device code of the GEMM kernel
 
 
+def strip_comments(src: str) -> str:
+    """C++ source without its comments and blank lines (the device code only)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip())
+
+
 def kernel_source_hash() -> str:
-    """Hash of the GEMM kernel's device code: DRAM counters recorded for another hash are stale."""
+    """Hash of the GEMM kernel's device code, comments excluded: DRAM counters recorded for
+    another hash are stale."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tiled_dense_gemm_tlg_b200", "csrc")
     for name in KERNEL_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -77,3 +77,12 @@ def test_nvml_sampler_keeps_the_timed_window():
     out = s.stop()
     assert out["samples"] == 3 and out["sm_mhz"] == 1500 and out["reasons"] == ["sw_power_cap"]
     assert out["sm_max_mhz"] == 1965 and out["power_w_median"] == 990.0
+
+
+def test_kernel_hash_ignores_comments_only():
+    import bench
+
+    code = "int f(int x) {\n  return x + 1;  // one more\n}\n/* block\n comment */\n"
+    assert bench.strip_comments(code) == bench.strip_comments(code.replace("one more", "plus one"))
+    assert bench.strip_comments(code) != bench.strip_comments(code.replace("x + 1", "x + 2"))
+    assert "//" not in bench.strip_comments(code) and "block" not in bench.strip_comments(code)

@@ -105,7 +105,7 @@ struct GemmParams {
   int c_plain;       // C cannot be written by TMA (base or row stride not 16-byte aligned)
   int bias_aligned;  // the bias may be read 16 bytes at a time
   // Fused epilogue (kernels built with kEpiFused): C = act(acc + bias[col]) + R[row, col].
-  int act;           // kActNone, kActRelu or kActGelu
+  int act;           // kActNone, kActRelu, kActGelu, kActSilu or kActGeluTanh
   const void *R;     // residual in C's type, or nullptr; may be C itself (same ldc)
   int64_t ldr;
   int r_vec;         // R's base and row stride are 16-byte aligned
