@@ -203,11 +203,16 @@ tlg_status tlg_gemm_ex(int64_t M, int64_t N, int64_t K,
  * no workspace.
  *
  * - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
- * - The first call on each device looks up the array's device address (with
- *   that device current) and may load the library's device code; make that
- *   first call before any stream capture.
+ * - Every call, split or not, first looks up the array's device address on
+ *   the current device (once per device; later calls reuse it).  The first
+ *   call on a device may also load the library's device code: make it before
+ *   any stream capture.
  * - A schedule needing more than 16 MiB of scratch gives TLG_ERR_UNSUPPORTED
  *   before anything is launched (tlg_gemm_workspace_size reports the need).
+ * - With split_k >= 2 and an A, B or C that TMA cannot describe (see
+ *   tlg_gemm_workspace_size_op), the aligned copies also go into the array,
+ *   after the split scratch, when they fit; otherwise the plain-load path
+ *   runs, as for tlg_gemm_ex with too small a workspace.
  * - Every call on a device shares the one array, which keeps what the last
  *   call left; each call clears the counters it needs on its stream first.
  *   Calls that overlap on the GPU (different streams, or different host

@@ -31,7 +31,8 @@ def tlg():
 
 
 def call_noalloc(tlg, A, B, bias, C, out, cfg):
-    """One raw C-ABI call of tlg_gemm_ex_noalloc on device tensors; returns the status."""
+    """One raw C-ABI call of tlg_gemm_ex_noalloc on device tensors (any row strides); returns
+    the status."""
     lib = tlg.raw_library()
     M, K = A.shape
     N = B.shape[1]
@@ -85,3 +86,65 @@ def test_scratch_beyond_the_limit_is_rejected(tlg):
     assert call_noalloc(tlg, A, A, None, C, "f16", cfg) == tlg.TLG_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert (C == 7.0).all()  # nothing was launched
+
+
+def odd_stride(host: torch.Tensor, pad_value: float) -> torch.Tensor:
+    """host on the device as a view whose row stride is one element longer than the row (not a
+    multiple of 16 bytes, so TMA cannot describe it); the extra column holds pad_value."""
+    rows, cols = host.shape
+    buf = torch.full((rows, cols + 1), pad_value, dtype=host.dtype, device="cuda")
+    view = buf[:, :cols]
+    view.copy_(host.to("cuda"))
+    return view
+
+
+def test_odd_strides_put_aligned_copies_beside_the_split_scratch(tlg):
+    # Every row stride odd and a forced split: the call copies A, B and C into aligned layouts
+    # in the same static array, after the split partials and counters.  Two calls in a row.
+    M, N, K, out = 600, 520, 2000, "f32"
+    cfg = {"cta_group": 1, "block_n": 128, "split_k": 4}
+    for i in range(2):
+        A, B, _ = wl.make_operands(M, N, K, "normal025", bias=False, seed=200 + i)
+        dA, dB = odd_stride(A, float("nan")), odd_stride(B, float("nan"))
+        C = odd_stride(torch.zeros((M, N), dtype=torch.float32), float("nan"))
+        C[:] = float("nan")
+        assert dA.stride(0) == K + 1 and dB.stride(0) == N + 1 and C.stride(0) == N + 1
+        need = tlg.tlg_gemm_workspace_size_op(dA, dB, C, "N", "N", out, config=cfg)
+        assert need <= 16 << 20  # the copies fit in the static array beside the split scratch
+        assert call_noalloc(tlg, dA, dB, None, C, out, cfg) == tlg.TLG_OK
+        ws = tlg.tlg_workspace(need)
+        ref_gpu = odd_stride(torch.zeros((M, N), dtype=torch.float32), float("nan"))
+        tlg.tlg_gemm_op(dA, dB, "N", "N", None, ref_gpu, out=out, config=cfg, workspace=ws)
+        torch.cuda.synchronize()
+        got = C.double().cpu().numpy()
+        ok, worst, idx = oracle.within_tolerance(got, ref_gpu.double().cpu().numpy(), out)
+        assert ok, f"vs tlg_gemm_op with a workspace: worst err/bound {worst:.3g} at {idx}"
+        ok, worst, idx = oracle.within_tolerance(got, oracle.gemm(A, B), out)
+        assert ok, f"vs oracle: worst err/bound {worst:.3g} at {idx}"
+        # the padding column of C (between rows) is untouched
+        pad = C.as_strided((M,), (N + 1,), storage_offset=C.storage_offset() + N)
+        assert torch.isnan(pad).all()
+    rc, code = tlg.tlg_device_error(clear=True)
+    assert rc == 0 and code == 0, hex(code)
+
+
+def test_a_call_allocates_nothing(tlg):
+    # Everything the calls touch exists before the first one; a warm-up call does the one-time
+    # set-up (the array's address, kernel attributes).  A later call must change neither the
+    # device's free memory nor torch's allocator.
+    M, N, K, out = 1024, 768, 1000, "f16"
+    cfg = {"cta_group": 2, "block_n": 256, "split_k": 3}
+    A, B, bias = wl.make_operands(M, N, K, "normal025", bias=True, seed=300)
+    dA, dB, dbias = A.cuda(), B.cuda(), bias.cuda()
+    C = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    assert call_noalloc(tlg, dA, dB, dbias, C, out, cfg) == tlg.TLG_OK
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    for _ in range(3):
+        assert call_noalloc(tlg, dA, dB, dbias, C, out, cfg) == tlg.TLG_OK
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
+    ok, worst, idx = oracle.within_tolerance(C.double().cpu().numpy(),
+                                             oracle.gemm(A, B, bias=bias, relu=True), out)
+    assert ok, f"vs oracle: worst err/bound {worst:.3g} at {idx}"

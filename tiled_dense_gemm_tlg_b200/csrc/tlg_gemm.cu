@@ -710,10 +710,14 @@ tlg_status check_args(int64_t M, int64_t N, int64_t K, bool at, const void *A, i
   return TLG_OK;
 }
 
-// ws/ws_bytes: scratch for the split-K tail (nullptr/0: none).
+// ws/ws_bytes: scratch for the split-K tail (nullptr/0: none).  static_ws: ws is the
+// library's own static scratch (tlg_gemm_ex_noalloc), whose split-K counters hold whatever
+// the last call left: they are cleared on the stream just before this call's first launch,
+// and a schedule that needs more scratch than it has is TLG_ERR_UNSUPPORTED.
 tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, int64_t lda,
                      bool bt, const void *B, int64_t ldb, const Epi &e, void *C, int64_t ldc,
-                     tlg_out out, const tlg_config *req, void *ws, size_t ws_bytes, void *stream) {
+                     tlg_out out, const tlg_config *req, void *ws, size_t ws_bytes, void *stream,
+                     bool static_ws = false) {
   const tlg_status hs = check_args(M, N, K, at, A, lda, bt, B, ldb, e, C, ldc, out);
   const void *bias = e.bias;
   if (hs != TLG_OK || M == 0 || N == 0) return hs;
@@ -794,13 +798,19 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
     copy_base = round_up_sz(std::max<size_t>(rv.sched.workspace, kCounterBytes), kCopyAlign);
   }
   if (rs != TLG_OK) return rs;
-  if (rv.sched.workspace > ws_bytes) return TLG_ERR_INVALID_ARG;  // a forced split needs scratch
+  if (rv.sched.workspace > ws_bytes)  // a forced split needs scratch
+    return static_ws ? TLG_ERR_UNSUPPORTED : TLG_ERR_INVALID_ARG;
   const size_t c_off = copy_base + (copy_ab ? cp.ab_bytes() : 0);
   if (cp.c && ws != nullptr && c_off + cp.c_bytes <= ws_bytes) copy_c = true;
   const bool c_plain = cp.c && !copy_c;
   char *wsb = static_cast<char *>(ws);
   const void *A_use = A, *B_use = B;
   int64_t lda_use = lda, ldb_use = ldb;
+  if (static_ws && rv.sched.split > 1 &&
+      cudaMemsetAsync(ws, 0, kCounterBytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return TLG_ERR_CUDA;
+  }
   if (copy_ab) {
     size_t off = copy_base;
     CopyJob jobs[2];
@@ -1030,28 +1040,18 @@ tlg_status tlg_gemm_ex_noalloc(int64_t M, int64_t N, int64_t K, const void *A, i
   Epi e;
   const tlg_status es = legacy_epilogue(out, epilogue, bias, &e);
   if (es != TLG_OK) return es;
+  // Looked up on every call, split or not, so that a device's first call does it.
+  void *scratch = nullptr;
+  const tlg_status ss = static_scratch(&scratch);
+  if (ss != TLG_OK) return ss;
   const bool split = config != nullptr && config->split_k >= 2;
   if (!split)  // no scratch needed: exactly tlg_gemm_ex without a workspace
     return gemm_impl(M, N, K, false, A, lda, false, B, ldb, e, C, ldc, out, config, nullptr, 0,
                      stream);
-  // Reject a schedule whose scratch would not fit before touching anything.
-  if (M > 0 && N > 0 && K > 0) {
-    Resolved rv;
-    const tlg_status rs = resolve_public(M, N, K, out, epilogue, config, SIZE_MAX, &rv);
-    if (rs != TLG_OK) return rs;
-    if (rv.sched.workspace > kStaticScratchBytes) return TLG_ERR_UNSUPPORTED;
-  }
-  void *scratch = nullptr;
-  const tlg_status ss = static_scratch(&scratch);
-  if (ss != TLG_OK) return ss;
-  // The counters must start at zero; the array keeps whatever the last call left.
-  if (M > 0 && N > 0 && K > 0 &&
-      cudaMemsetAsync(scratch, 0, kCounterBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-    cudaGetLastError();
-    return TLG_ERR_CUDA;
-  }
+  // gemm_impl rejects a schedule that needs more scratch than the array holds before it
+  // launches anything, and clears the counters just before its first launch.
   return gemm_impl(M, N, K, false, A, lda, false, B, ldb, e, C, ldc, out, config, scratch,
-                   kStaticScratchBytes, stream);
+                   kStaticScratchBytes, stream, true);
 }
 
 tlg_status tlg_gemm_workspace_size(int64_t M, int64_t N, int64_t K, tlg_out out,
