@@ -294,6 +294,11 @@ def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float)
     return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
+def ms_per_step_est(per_step_ms) -> float:
+    """A step's device time, for sizing a run of a given length."""
+    return statistics.median(per_step_ms)
+
+
 def all_workloads():
     return {**wl.WORKLOADS, **wl.EPILOGUE_WORKLOADS}
 
@@ -393,6 +398,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layout", default="NN", choices=["NN", "NT", "TN", "TT"],
                     help="op(A), op(B): T = that operand is stored transposed (tlg_gemm_op)")
+    ap.add_argument("--sustained-s", type=float, default=3.0,
+                    help="seconds of back-to-back calls (inputs rotated over buffer sets larger than L2) "
+                         "timed after the burst steps, with the SM clock sampled; 0 skips it")
     ap.add_argument("--ld-pad", type=int, default=0,
                     help="extra elements in every row stride (odd: strides TMA cannot describe; "
                          "the bench passes the workspace the size query asks for, so the call "
@@ -488,6 +496,29 @@ def main(argv=None):
         else:
             plain_step()
 
+    def gemm_into(a, b, bias_, r_, c, st):
+        """The timed call on one set of device buffers, on stream st."""
+        if fused:
+            tlg.tlg_gemm_fused(a, b, args.layout[0], args.layout[1], bias=bias_, activation=w.act,
+                               residual=r_, C=c, out=w.out, config=override, workspace=ws, stream=st)
+        elif use_op:
+            tlg.tlg_gemm_op(a, b, args.layout[0], args.layout[1], bias_, c, out=w.out, config=override,
+                            workspace=ws, stream=st)
+        elif use_ex:
+            tlg.tlg_gemm_ex(a, b, bias_, c, out=w.out, config=override, workspace=ws, stream=st)
+        elif w.bias_relu:
+            tlg.tlg_gemm_bias_relu_f16(a, b, bias_, c, stream=st)
+        elif w.out == "f16":
+            tlg.tlg_gemm_f16f16(a, b, c, stream=st)
+        else:
+            tlg.tlg_gemm_f16f32(a, b, c, stream=st)
+
+    def new_buffer_set():
+        """Another device copy of the step's operands and output, same layout."""
+        return (padded(A, args.ld_pad), padded(B, args.ld_pad), bias.to(dev) if bias is not None else None,
+                padded(R, args.ld_pad) if R is not None else None,
+                padded(torch.empty((w.M, w.N), dtype=dC.dtype), args.ld_pad))
+
     def timed(fn, n):
         """Per-step device milliseconds of n calls, each after an untimed L2 flush."""
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -549,6 +580,49 @@ def main(argv=None):
     value = job_throughput(w.flops, args.steps, world, max_ms)
     ms_per_step = max_ms / args.steps
 
+    # ---- sustained rate: the same call back to back for a few seconds, with no flush in between;
+    # the inputs rotate over enough buffer sets that together they exceed the 126 MB L2, so each
+    # call still reads its operands from HBM.  The SM clock is sampled over the window: under the
+    # 1000 W cap a long run settles at a lower clock than the short burst above.
+    sustained = None
+    if args.sustained_s > 0:
+        set_bytes = A.numel() * 2 + B.numel() * 2 + dC.numel() * dC.element_size() + (
+            R.numel() * R.element_size() if R is not None else 0)
+        sets = [(dA, dB, dbias, dR, dC)]
+        while len(sets) < 8 and len(sets) * set_bytes < 3 * (126 << 20):
+            sets.append(new_buffer_set())
+        n = max(len(sets), int(args.sustained_s * 1e3 / max(ms_per_step_est(per_step_ms), 1e-3)))
+        for i in range(len(sets)):
+            gemm_into(*sets[i], stream)
+        torch.cuda.synchronize(dev)
+        try:
+            sclk = NvmlClockSampler(nvsmi_id(dev))
+        except Exception:
+            sclk = ClockSampler(nvsmi_id(dev))
+        sclk.start()
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sclk.mark_begin()
+        e0.record(stream)
+        for i in range(n):
+            gemm_into(*sets[i % len(sets)], stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        sclk.mark_end()
+        sc = sclk.stop()
+        s_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        rc, code = tlg.tlg_device_error(clear=True)
+        if rc != 0:
+            raise SystemExit(f"device error word {code:#x} during the sustained run")
+        s_val = w.flops * n * world / (s_ms * 1e-3) / 1e12
+        sustained = {"value": s_val, "unit": UNIT, "seconds": s_ms * 1e-3, "calls": n,
+                     "buffer_sets": len(sets), "ms_per_call": s_ms / n, "clocks": sc}
+        if sc:
+            sustained["mcycles_per_call"] = s_ms / n * sc["sm_mhz"] * 1e-3
+            sustained["frac_of_clock_peak"] = s_val / world / (148 * 8192 * sc["sm_mhz"] * 1e6 / 1e12)
+        del sets
+
     # ---- end to end through the public API: pinned host inputs -> device -> GEMM -> pinned host output.
     # Every step copies its inputs in and its result out inside the timed region.  The steps are
     # pipelined the way a host-fed job would run them: two device buffer sets, the uploads on one
@@ -563,30 +637,10 @@ def main(argv=None):
         h2d = hA.numel() * 2 + hB.numel() * 2 + (hbias.numel() * 2 if hbias is not None else 0)
         h2d += hR.numel() * hR.element_size() if hR is not None else 0
         d2h = hC[0].numel() * hC[0].element_size()
-        bufs = [(dA, dB, dbias, dR, dC)]
-        bufs.append((padded(A, args.ld_pad), padded(B, args.ld_pad),
-                     bias.to(dev) if bias is not None else None,
-                     padded(R, args.ld_pad) if R is not None else None,
-                     padded(torch.empty((w.M, w.N), dtype=dC.dtype), args.ld_pad)))
+        bufs = [(dA, dB, dbias, dR, dC), new_buffer_set()]
         s_up, s_gemm, s_down = (torch.cuda.Stream(dev) for _ in range(3))
         ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("up", "gemm", "down")}
         used = [False, False]
-
-        def gemm_into(a, b, bias_, r_, c, st):
-            if fused:
-                tlg.tlg_gemm_fused(a, b, args.layout[0], args.layout[1], bias=bias_, activation=w.act,
-                                   residual=r_, C=c, out=w.out, config=override, workspace=ws, stream=st)
-            elif use_op:
-                tlg.tlg_gemm_op(a, b, args.layout[0], args.layout[1], bias_, c, out=w.out, config=override,
-                                workspace=ws, stream=st)
-            elif use_ex:
-                tlg.tlg_gemm_ex(a, b, bias_, c, out=w.out, config=override, workspace=ws, stream=st)
-            elif w.bias_relu:
-                tlg.tlg_gemm_bias_relu_f16(a, b, bias_, c, stream=st)
-            elif w.out == "f16":
-                tlg.tlg_gemm_f16f16(a, b, c, stream=st)
-            else:
-                tlg.tlg_gemm_f16f32(a, b, c, stream=st)
 
         def e2e_step(i):
             k = i % 2
@@ -675,6 +729,7 @@ def main(argv=None):
                                       else "plain loads/stores") + " (row strides not 16-byte multiples)"
                                      if (args.ld_pad * 2) % 16 else "TMA")),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "plain_entry_point": plain,
+        "sustained": sustained,
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clk,
         "per_step_ms": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
