@@ -705,6 +705,22 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
+    // The MMAs of accumulator half h (h = 0 with NH == 1) for the k-block in ring slot st.
+    auto issue_half = [&](int st, int h, bool first_kb) {
+      const uint32_t a0 = smem_u32(sA + st * Plan::kABytes);
+      const uint32_t bh = smem_u32(sB + st * Plan::kBBytes) + h * Plan::kHalfBBytes;
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((NH == 1 ? acc : h) * BN);
+#pragma unroll
+      for (int kk = 0; kk < kBK / 16; ++kk) {
+        // K-major: 16 k = 32 bytes along the swizzled row; MN-major: 16 k
+        // = 16 rows of 128 bytes, 64-element blocks 8192 bytes apart.
+        const uint64_t adesc = !AT ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
+                                   : smem_desc_sw128(a0 + kk * 16 * 128, 8192, 1024);
+        const uint64_t bdesc = !BT ? smem_desc_sw128(bh + kk * 16 * 128, 8192, 1024)
+                                   : smem_desc_sw128(bh + kk * 32, 16, 1024);
+        mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (!first_kb || kk > 0) ? 1u : 0u);
+      }
+    };
     for (int k = 0; k < n_work && ok; ++k) {
       const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
       if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
@@ -713,46 +729,63 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      bool half1_free = NH == 1;  // NH == 2: waited for just before its first MMA
+      // NH == 2: when this tile's first k-blocks land, the epilogue may still be draining
+      // half 1 of the previous tile.  Their half-0 MMAs then run ahead (up to the ring's
+      // depth, the slots held), and their half-1 MMAs follow in k order as soon as half 1
+      // is handed back; only then are the slots released.  Each half still sums its
+      // k-blocks in ascending order.
+      bool half1_free = NH == 1;
+      int pend = 0;        // k-blocks w.kb0 .. w.kb0 + pend - 1: half 0 issued, half 1 not yet
+      int pend_stage = 0;  // the ring slot of the first of them
+      auto half1_ready = [&]() {
+        tc_fence_after_sync();
+        half1_free = true;
+        int st = pend_stage;
+        for (int i = 0; i < pend; ++i) {
+          issue_half(st, 1, i == 0);
+          mma_commit<CG>(empty_bar(st));
+          if (++st == STAGES) st = 0;
+        }
+        pend = 0;
+      };
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        if (NH == 2 && !half1_free && pend == STAGES) {
+          // every slot holds a run-ahead k-block: nothing more can land before half 1 is free
+          if (!mbar_wait(tempty_bar(1), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
+                         &g_device_error)) {
+            ok = false;
+            break;
+          }
+          half1_ready();
+        }
         if (!mbar_wait(full_bar(stage), phase, abort_flag, p.limit_ns, kRoleMma,
                        &g_device_error)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t a0 = smem_u32(sA + stage * Plan::kABytes);
-        const uint32_t b0 = smem_u32(sB + stage * Plan::kBBytes);
+        if (NH == 2 && !half1_free && mbar_test_wait(tempty_bar(1), acc_phase ^ 1u)) half1_ready();
+        if (NH == 2 && !half1_free) {
+          if (pend == 0) pend_stage = stage;
+          issue_half(stage, 0, kb == w.kb0);
+          ++pend;
+        } else {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          if (NH == 2 && h == 1 && !half1_free) {
-            if (!mbar_wait(tempty_bar(1), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
-                           &g_device_error)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after_sync();
-            half1_free = true;
-          }
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((NH == 1 ? acc : h) * BN);
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            // K-major: 16 k = 32 bytes along the swizzled row; MN-major: 16 k
-            // = 16 rows of 128 bytes, 64-element blocks 8192 bytes apart.
-            const uint64_t adesc = !AT ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
-                                       : smem_desc_sw128(a0 + kk * 16 * 128, 8192, 1024);
-            const uint32_t bh = b0 + h * Plan::kHalfBBytes;
-            const uint64_t bdesc = !BT ? smem_desc_sw128(bh + kk * 16 * 128, 8192, 1024)
-                                       : smem_desc_sw128(bh + kk * 32, 16, 1024);
-            mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (kb > w.kb0 || kk > 0) ? 1u : 0u);
-          }
+          for (int h = 0; h < NH; ++h) issue_half(stage, h, kb == w.kb0);
+          mma_commit<CG>(empty_bar(stage));
         }
-        if (!ok) break;
-        mma_commit<CG>(empty_bar(stage));
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
+      }
+      if (ok && NH == 2 && !half1_free) {
+        // a tile shorter than the epilogue's half 1: finish its half-1 MMAs now
+        if (!mbar_wait(tempty_bar(1), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
+                       &g_device_error))
+          ok = false;
+        else
+          half1_ready();
       }
       if (!ok) break;
       mma_commit<CG>(tfull_bar(acc));
