@@ -144,6 +144,16 @@ typedef enum tlg_epilogue { TLG_EPI_NONE = 0, TLG_EPI_BIAS_RELU = 1 } tlg_epilog
  *                 finishing (programmatic dependent launch); it reads and
  *                 writes global memory only after that kernel has completed.
  *                 0 (default) = ordinary stream order.
+ *   k_split     : 1 = each tile's whole K range is summed by one CTA (or CTA
+ *                 pair); 2 or 4 = a cluster of that many one-CTA tiles'
+ *                 CTAs shares every tile, each summing a slice of its
+ *                 k-blocks, and the partial sums are added in slice order
+ *                 through distributed shared memory (no workspace, so the
+ *                 plain entry points use it too).  Built for block_n 128
+ *                 (k_split 2) and 256 (k_split 2 or 4), untransposed operands
+ *                 that TMA can describe, at least k_split k-blocks of 64, and
+ *                 no split_k tail.  0 = automatic: chosen where few tiles
+ *                 would leave most SMs idle (small or short-K shapes).
  * A combination the library does not provide gives TLG_ERR_UNSUPPORTED.
  */
 typedef struct tlg_config {
@@ -154,6 +164,7 @@ typedef struct tlg_config {
     int32_t max_ctas;
     int32_t split_k;
     int32_t overlap_prev;
+    int32_t k_split;
 } tlg_config;
 
 /*

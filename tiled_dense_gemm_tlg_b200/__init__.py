@@ -56,7 +56,7 @@ EXPORTED = ("tlg_gemm_f16f32", "tlg_gemm_f16f16", "tlg_gemm_bias_relu_f16", "tlg
 class tlg_config(ctypes.Structure):
     _fields_ = [("block_n", ctypes.c_int32), ("stages", ctypes.c_int32), ("cta_group", ctypes.c_int32),
                 ("raster_group", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("split_k", ctypes.c_int32), ("overlap_prev", ctypes.c_int32)]
+                ("split_k", ctypes.c_int32), ("overlap_prev", ctypes.c_int32), ("k_split", ctypes.c_int32)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

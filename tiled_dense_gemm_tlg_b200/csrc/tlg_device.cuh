@@ -112,6 +112,39 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
   }
 }
 
+// The same wait with acquire semantics at cluster scope: the phase was completed by
+// release-arrives of threads in other CTAs of the cluster, and their writes to this
+// CTA's shared memory (made before they arrived) are visible once it returns true.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity,
+                                                      uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+static __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                     volatile uint32_t *abort_flag,
+                                                     uint64_t limit_ns, uint32_t role,
+                                                     uint32_t *err_word) {
+  if (mbar_try_wait_cluster(bar, parity, 0u)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity, kWaitSuspendNs)) return true;
+    if (abort_flag != nullptr && *abort_flag != 0u) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(err_word, kErrTimeout | role);
+      if (abort_flag != nullptr) *abort_flag = 1u;
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t *abort_flag, uint64_t limit_ns,
                                           uint32_t role, uint32_t *err_word) {
@@ -241,6 +274,23 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile(
       "barrier.cluster.arrive.release.aligned;\n\t"
       "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 16 bytes to a shared::cluster address (this CTA's or a peer's shared memory).
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
+               "r"(c), "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {

@@ -97,6 +97,8 @@ struct KernelCfg {
   double eff;         // sustained fraction of the MMA peak, relative (ranks tile shapes)
   double exposed_kb;  // k-blocks per tile the main loop waits for the epilogue
   bool plain_loads;   // also built with the plain-load path (operands TMA cannot describe)
+  int ks;             // CTAs of a cluster sharing each tile's K range (1: none)
+  double reduce_kb;   // k-split: the reduction through distributed shared memory, in k-blocks
 };
 
 // Kernel variants the library is built with.  A tile is 128*cta_group rows by
@@ -110,9 +112,21 @@ struct KernelCfg {
 // its single accumulator leaves part of each epilogue exposed (exposed_kb).
 // Its two numbers fit both measured points at equal wave fill: 0.93x the pair
 // 256 tile at 4096^3 (64 k-blocks) and 1.05x at 8192^3 (128 k-blocks).
-constexpr KernelCfg kBuilt[] = {{1, 64, 8, 0.35, 0, true},   {1, 128, 6, 0.60, 0, false},
-                                {1, 256, 4, 0.90, 0, false},  {2, 128, 8, 0.60, 0, false},
-                                {2, 256, 6, 1.00, 0, true},   {2, 512, 4, 1.20, 19, false}};
+// The last three split each tile's K range over a cluster of 2 or 4 CTAs and
+// reduce the partial sums through distributed shared memory (their receive
+// buffers leave room for fewer ring stages); they are built for untransposed
+// TMA operands.  A CTA of such a cluster streams only its share of the
+// k-blocks, so a shape with few tiles keeps more SMs busy, and the wider tile
+// reads fewer operand bytes per FLOP than the 128 x 64 tile that would
+// otherwise spread it.  Their reduce_kb is the measured cost of the exchange,
+// in k-blocks of their tile (B200, one tile per cluster, fp32 C): about 1.3 us
+// for 32 KB per CTA each way, 2-5 us for 64-96 KB.  So they pay off only where
+// K is long next to M x N, not at 256^3 or 1024^3.
+constexpr KernelCfg kBuilt[] = {{1, 64, 8, 0.35, 0, true, 1, 0},   {1, 128, 6, 0.60, 0, false, 1, 0},
+                                {1, 256, 4, 0.90, 0, false, 1, 0},  {2, 128, 8, 0.60, 0, false, 1, 0},
+                                {2, 256, 6, 1.00, 0, true, 1, 0},   {2, 512, 4, 1.20, 19, false, 1, 0},
+                                {1, 128, 5, 0.60, 0, false, 2, 6.0}, {1, 256, 2, 0.90, 0, false, 2, 12.0},
+                                {1, 256, 2, 0.90, 0, false, 4, 12.0}};
 constexpr int kNumBuilt = sizeof(kBuilt) / sizeof(kBuilt[0]);
 static_assert(kNumBuilt == kNumVariants, "one launcher table entry per built variant");
 
@@ -203,7 +217,7 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
   if (req != nullptr) r = *req;
   if (r.raster_group < 0 || r.raster_group > 64 || r.max_ctas < 0 || r.split_k < 0 ||
       r.split_k > 16 || r.stages < 0 || r.block_n < 0 || r.cta_group < 0 ||
-      (r.overlap_prev != 0 && r.overlap_prev != 1))
+      (r.overlap_prev != 0 && r.overlap_prev != 1) || r.k_split < 0 || r.k_split > 16)
     return TLG_ERR_UNSUPPORTED;
   double best_cost = 0;
   bool found = false;
@@ -214,11 +228,14 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
     if (r.block_n != 0 && r.block_n != k.block_n) continue;
     if (r.stages != 0 && r.stages != k.stages) continue;
     if (plain && !k.plain_loads) continue;
+    if (r.k_split != 0 && r.k_split != k.ks) continue;
+    // a k-split: untransposed TMA operands, at least one k-block per CTA, no split tail
+    if (k.ks > 1 && (at || bt || plain || num_kb < k.ks || r.split_k >= 2)) continue;
     shape_exists = true;
     int resident = 0;
     const tlg_status us = fns_for(i, f16, ek, at, bt, plain).units(dev, sms, &resident);
     if (us != TLG_OK) return us;
-    if (r.max_ctas > 0) resident = std::max(1, std::min(resident, r.max_ctas / k.cta_group));
+    if (r.max_ctas > 0) resident = std::max(1, std::min(resident, r.max_ctas / (k.cta_group * k.ks)));
     const int64_t tile_m = 128 * k.cta_group;
     const int64_t tiles = ((M + tile_m - 1) / tile_m) * ((N + k.block_n - 1) / k.block_n);
     // Automatic choice (split_k == 0): every tile whole, or, when the caller's
@@ -228,14 +245,16 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
     // 4096^3 (3.46 waves) ran 4.5 % faster, while a split with no whole wave
     // before it lost at 1024^3, where the fix-up is exposed.
     const int split_lo = r.split_k == 0 ? 1 : r.split_k;
-    const int split_hi = r.split_k == 0 ? (ws_bytes > 0 ? 4 : 1) : r.split_k;
+    const int split_hi = r.split_k == 0 && k.ks == 1 ? (ws_bytes > 0 ? 4 : 1) : split_lo;
+    // k-blocks one CTA of the tile's group sums (its slice, with a k-split)
+    const int kb_unit = (num_kb + k.ks - 1) / k.ks;
     for (int split = split_lo; split <= split_hi; ++split) {
       Schedule sch;
-      if (!plan(tiles, resident, num_kb, split, k.cta_group, k.block_n, &sch)) continue;
+      if (!plan(tiles, resident, kb_unit, split, k.cta_group, k.block_n, &sch)) continue;
       if (r.split_k == 0 && split > 1 && (sch.dp_tiles == 0 || sch.workspace > ws_bytes)) continue;
       // the busiest unit's tile count, each tile paying the exposed part of its epilogue
       const double per_unit_tiles = static_cast<double>((tiles + sch.units - 1) / sch.units);
-      const double cost = (sch.cost + per_unit_tiles * k.exposed_kb) *
+      const double cost = (sch.cost + per_unit_tiles * (k.exposed_kb + k.reduce_kb)) *
                           static_cast<double>(tile_m * k.block_n) / (k.cta_group * k.eff);
       if (!found || cost < best_cost * 0.999) {
         found = true;
@@ -245,12 +264,13 @@ tlg_status resolve(int dev, int sms, int64_t M, int64_t N, int64_t K, bool f16, 
         out->cfg.cta_group = k.cta_group;
         out->cfg.block_n = k.block_n;
         out->cfg.stages = k.stages;
+        out->cfg.k_split = k.ks;
       }
     }
   }
   if (!shape_exists || !found) return TLG_ERR_UNSUPPORTED;
   out->cfg.raster_group = r.raster_group != 0 ? r.raster_group : 8;
-  out->cfg.max_ctas = out->sched.units * out->cfg.cta_group;  // the CTAs the launch uses
+  out->cfg.max_ctas = out->sched.units * out->cfg.cta_group * out->cfg.k_split;  // CTAs launched
   out->cfg.split_k = out->sched.split;
   out->cfg.overlap_prev = r.overlap_prev;
   return TLG_OK;

@@ -62,8 +62,10 @@ static __device__ uint32_t g_device_error;
 // 128*CG rows by NH*BN columns (BN = the MMA's N; NH = 1, or 2 for a tile of
 // two MMA halves that fills TMEM); each CTA stages its own 128 rows of A and
 // its own BN/CG columns of each half of B per k-block, plus two 4 KB output
-// boxes per epilogue warp.
-template <int CG, int BN, int STAGES, int NH = 1>
+// boxes per epilogue warp.  With a cluster k-split (KS > 1 CTAs share one
+// tile's K range) each CTA also receives, for the BN/KS columns it finishes,
+// the fp32 partial sums of its KS - 1 peers.
+template <int CG, int BN, int STAGES, int NH = 1, int KS = 1>
 struct SmemPlan {
   static constexpr int kBNc = BN / CG;  // B columns of one MMA half held by one CTA
   static constexpr uint32_t kABytes = kBM * kBK * 2;
@@ -72,14 +74,21 @@ struct SmemPlan {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kOutOffset = STAGES * kStageBytes;
   static constexpr uint32_t kOutBytes = kEpiWarps * 2 * kStageOutBytes;
-  static constexpr uint32_t kBarOffset = kOutOffset + kOutBytes;
-  static constexpr uint32_t kNumBars = 2 * STAGES + 4 + 1;  // full, empty, tmem full/empty x2, drain
+  static constexpr int kOwnCols = BN / KS;  // columns of a tile one CTA of a k-split finishes
+  static constexpr uint32_t kRecvSlotBytes = kBM * kOwnCols * 4;  // one peer's fp32 partial of them
+  static constexpr uint32_t kRecvOffset = kOutOffset + kOutBytes;
+  static constexpr uint32_t kRecvBytes = (KS - 1) * kRecvSlotBytes;
+  static constexpr uint32_t kBarOffset = kRecvOffset + kRecvBytes;
+  // full, empty, tmem full/empty x2, drain; with a k-split also recv-full and send-free
+  static constexpr uint32_t kNumBars = 2 * STAGES + 4 + 1 + (KS > 1 ? 2 : 0);
   static constexpr uint32_t kMiscOffset = kBarOffset + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOffset + 16;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack to align the base to 1024
   static constexpr uint32_t kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
   static_assert(kBNc % 64 == 0, "each CTA's B slice must be whole 64-column swizzle blocks");
   static_assert(kTmemCols <= 512, "two accumulators must fit in TMEM");
+  static_assert(KS == 1 || (CG == 1 && NH == 1 && kOwnCols % 64 == 0),
+                "a k-split is built for one-CTA tiles whose CTAs each finish whole 64-column pieces");
   static_assert(kDynamicBytes <= 232448, "shared memory per CTA exceeded");
 };
 
@@ -535,19 +544,28 @@ __device__ __forceinline__ uint32_t mnmajor_offset(int mn, int k) {
 // LSU: the operands are loaded by kLoaderWarps extra warps with 2-byte global
 // loads into the same swizzled shared-memory layouts, for strides and bases
 // the TMA unit cannot describe; the tensor-core pipeline is unchanged.
+//
+// KS > 1 (one-CTA tiles only): a cluster of KS CTAs shares every tile, CTA s
+// summing k-blocks [s*kb/KS, (s+1)*kb/KS).  The partial sums are reduced
+// through distributed shared memory: each CTA finishes BN/KS of the tile's
+// columns, receiving the other CTAs' fp32 partials of them into its own shared
+// memory, and adds all KS slices in slice order before the epilogue.  No
+// global scratch is needed, and the result does not depend on timing.
 template <int CG, int BN, int STAGES, bool OUT_F16, int EK, int NH = 1, bool AT = false,
-          bool BT = false, bool LSU = false>
+          bool BT = false, bool LSU = false, int KS = 1>
 __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
-  using Plan = SmemPlan<CG, BN, STAGES, NH>;
+  using Plan = SmemPlan<CG, BN, STAGES, NH, KS>;
   constexpr int kTileM = kBM * CG;
   constexpr int kTileN = BN * NH;
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
   static_assert(NH == 1 || NH == 2, "one accumulator per tile, or two halves");
   static_assert(!LSU || NH == 1, "the plain-load path is built for one-accumulator tiles");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
+  static_assert(KS == 1 || (CG == 1 && NH == 1 && !LSU), "the k-split is built for one-CTA TMA tiles");
+  constexpr bool kCluster = CG == 2 || KS > 1;  // CTAs of a work unit form a cluster
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -560,21 +578,37 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  // k-split: this CTA's receive buffer is full (every peer wrote and arrived) / every
+  // peer has consumed this CTA's partials from its own receive buffer.
+  const uint32_t recv_full_bar = bar0 + 8u * (2 * STAGES + 5);
+  const uint32_t send_free_bar = bar0 + 8u * (2 * STAGES + 6);
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + Plan::kMiscOffset);
   uint32_t *tmem_holder = misc;
   volatile uint32_t *abort_flag = misc + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Work unit = one tile per CTA group: a CTA (CG == 1) or a cluster of two (CG == 2).
+  // Work unit = one tile per CTA group: a CTA (CG == 1), a cluster of two (CG == 2), or a
+  // cluster of KS CTAs that split each tile's K range.
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
-  const int unit = (CG == 2) ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
-  const int num_units = (CG == 2) ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+  const int kslice = (KS > 1) ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit = kCluster ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int num_units = kCluster ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
   const bool leader = rank == 0;
   const int num_m = (p.M + kTileM - 1) / kTileM;
   const int num_n = (p.N + kTileN - 1) / kTileN;
   const int num_kb = (p.K + kBK - 1) / kBK;
   const int n_work = work_count(p, unit, num_units);
+  // The k-th work item of this unit; with a k-split, this CTA's slice of its k-blocks
+  // (the host guarantees at least KS k-blocks, so no slice is empty).
+  auto item = [&](int k) {
+    WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+    if constexpr (KS > 1) {
+      w.kb0 = static_cast<int>(static_cast<int64_t>(kslice) * num_kb / KS);
+      w.kb1 = static_cast<int>(static_cast<int64_t>(kslice + 1) * num_kb / KS);
+    }
+    return w;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -586,6 +620,10 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       mbar_init(tempty_bar(a), kEpiWarps * CG);  // one arrive per epilogue warp of each CTA
     }
     mbar_init(drain_bar, 1);
+    if constexpr (KS > 1) {
+      mbar_init(recv_full_bar, (KS - 1) * 32 * kEpiWarps);  // every epilogue thread of each peer
+      mbar_init(send_free_bar, (KS - 1) * 32 * kEpiWarps);
+    }
     *abort_flag = 0u;
     fence_mbar_init();
     if constexpr (!LSU) {
@@ -600,8 +638,8 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
   }
   tc_fence_before_sync();
   __syncwarp();
-  if constexpr (CG == 2)
-    cluster_sync_all();  // both CTAs' barriers exist before either signals the other
+  if constexpr (kCluster)
+    cluster_sync_all();  // every CTA's barriers exist before any other signals them
   else
     __syncthreads();
   tc_fence_after_sync();
@@ -619,7 +657,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     uint32_t issued_mask = 0, issued_parity = 0;
     bool ok = true;
     for (int k = 0; k < n_work && ok; ++k) {
-      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+      const WorkItem w = item(k);
       const int a_row = w.mb * kTileM + static_cast<int>(rank) * kBM;
       const int b_col = w.nb * kTileN + static_cast<int>(rank) * Plan::kBNc;
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
@@ -722,7 +760,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       }
     };
     for (int k = 0; k < n_work && ok; ++k) {
-      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+      const WorkItem w = item(k);
       if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
                      &g_device_error)) {
         ok = false;
@@ -812,7 +850,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int k = 0; k < n_work && ok; ++k) {
-      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+      const WorkItem w = item(k);
       const int a_row = w.mb * kTileM + static_cast<int>(rank) * kBM;
       const int b_col = w.nb * kTileN + static_cast<int>(rank) * Plan::kBNc;
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
@@ -983,8 +1021,106 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       }
     };
 
+    // k-split (KS > 1): the reduction of one tile through distributed shared memory.
+    // Receive buffer of a CTA: one slot per peer (in rank order, skipping itself); in a
+    // slot, for epilogue warp w, 32-column chunk c and 4-column group g, lane l's 16
+    // bytes sit at ((w * kOwn / 32 + c) * 8 + g) * 512 + l * 16, so each warp-wide
+    // 16-byte store or load covers 512 contiguous bytes.
+    uint32_t recv_parity = 0, free_parity = 0;
+    auto ks_tile = [&](const WorkItem &w, int box_row0, const BiasSlice<kCPL> &bias,
+                       EpiIn<kPrefR> &in) -> bool {
+      constexpr int kOwn = Plan::kOwnCols;
+      const uint32_t recv0 = smem_u32(smem + Plan::kRecvOffset);
+      const uint32_t tmem_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                static_cast<uint32_t>(acc * BN);
+      const uint32_t warp_off = static_cast<uint32_t>(quarter * (kOwn / 32)) * 4096u +
+                                static_cast<uint32_t>(lane) * 16u;
+      // 1. This CTA's partial of every peer's columns, into that peer's receive buffer,
+      //    once every peer has consumed the previous tile's.
+      if (!mbar_wait_cluster(send_free_bar, free_parity ^ 1u, abort_flag, p.limit_ns,
+                             kRoleEpilogue, &g_device_error))
+        return false;
+      free_parity ^= 1u;
+#pragma unroll 1
+      for (int q = 0; q < KS; ++q) {
+        if (q == kslice) continue;
+        const uint32_t dst = mapa_shared(recv0, static_cast<uint32_t>(q)) +
+                             static_cast<uint32_t>(kslice < q ? kslice : kslice - 1) *
+                                 Plan::kRecvSlotBytes +
+                             warp_off;
+#pragma unroll 1
+        for (int c = 0; c < kOwn; c += 32) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_load_32cols(tmem_row + static_cast<uint32_t>(q * kOwn + c), r);
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            st_cluster_v4(dst + static_cast<uint32_t>(c / 32) * 4096u + g * 512u, r[4 * g],
+                          r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+        }
+        mbar_arrive_cluster(mapa_shared(recv_full_bar, static_cast<uint32_t>(q)));
+      }
+      // 2. This CTA's own columns: wait for the peers' partials, add the KS slices in
+      //    slice order, then the epilogue and the store of each 64-column piece.
+      if (!mbar_wait_cluster(recv_full_bar, recv_parity, abort_flag, p.limit_ns, kRoleEpilogue,
+                             &g_device_error))
+        return false;
+      recv_parity ^= 1u;
+#pragma unroll 1
+      for (int tc = 0; tc < kOwn; tc += 64) {
+        const int tcol = kslice * kOwn + tc;  // column within the tile
+        const int col0 = w.nb * kTileN + tcol;
+        uint32_t ra[32], rb[32];
+        __syncwarp();
+        tmem_load_2x32cols(tmem_row + static_cast<uint32_t>(tcol), ra, rb);
+        if (tc + 64 >= kOwn) {
+          // last read of this accumulator: hand it back to the MMA warp
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(acc));
+        }
+        if (box_row0 >= p.M || col0 >= p.N) continue;  // the whole 32 x 64 piece is clipped
+        float va[32], vb[32];
+#pragma unroll 1
+        for (int sl = 0; sl < KS; ++sl) {
+          if (sl == kslice) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              va[j] = sl == 0 ? __uint_as_float(ra[j]) : va[j] + __uint_as_float(ra[j]);
+              vb[j] = sl == 0 ? __uint_as_float(rb[j]) : vb[j] + __uint_as_float(rb[j]);
+            }
+          } else {
+            const uint32_t src = recv0 +
+                                 static_cast<uint32_t>(sl < kslice ? sl : sl - 1) * Plan::kRecvSlotBytes +
+                                 warp_off + static_cast<uint32_t>(tc / 32) * 4096u;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const uint4 xa = ld_shared_v4(src + g * 512u);
+              const uint4 xb = ld_shared_v4(src + 4096u + g * 512u);
+              const float fa[4] = {__uint_as_float(xa.x), __uint_as_float(xa.y), __uint_as_float(xa.z),
+                                   __uint_as_float(xa.w)};
+              const float fb[4] = {__uint_as_float(xb.x), __uint_as_float(xb.y), __uint_as_float(xb.z),
+                                   __uint_as_float(xb.w)};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                va[4 * g + e] = sl == 0 ? fa[e] : va[4 * g + e] + fa[e];
+                vb[4 * g + e] = sl == 0 ? fb[e] : vb[4 * g + e] + fb[e];
+              }
+            }
+          }
+        }
+        const int next_col0 = (tc + 64 < kOwn && col0 + 64 < p.N) ? col0 + 64 : -1;
+        emit64(va, vb, box_row0, col0, tcol, bias, in, next_col0);
+      }
+      // Every read of the receive buffer is done: the peers may write it again.
+#pragma unroll 1
+      for (int q = 0; q < KS; ++q)
+        if (q != kslice) mbar_arrive_cluster(mapa_shared(send_free_bar, static_cast<uint32_t>(q)));
+      return true;
+    };
+
     for (int k = 0; k < n_work; ++k) {
-      const WorkItem w = work_item(p, k, unit, num_units, num_m, num_n, num_kb);
+      const WorkItem w = item(k);
       const int box_row0 = w.mb * kTileM + box_row0_in_tile;
       // The tile's bias and the first piece's residual load while the main
       // loop still runs.
@@ -994,8 +1130,9 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         if (p.bias != nullptr && w.nb * kTileN < p.N) load_bias_slice<kCPL>(p, w.nb * kTileN, lane, bias);
       }
       if constexpr (kPrefR) {
-        if (w.tail < 0 && box_row0 < p.M && w.nb * kTileN < p.N)
-          epi_prefetch<kPrefR>(p, box_row0 + lane, w.nb * kTileN, in);
+        const int first_col = w.nb * kTileN + (KS > 1 ? kslice * Plan::kOwnCols : 0);
+        if (w.tail < 0 && box_row0 < p.M && first_col < p.N)
+          epi_prefetch<kPrefR>(p, box_row0 + lane, first_col, in);
       }
       // This wait spans the tile's whole main loop, so its limit grows with the
       // tile's k-blocks (20 us each, far above a k-block's time on any built
@@ -1006,6 +1143,9 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
                      &g_device_error))
         break;
       tc_fence_after_sync();
+      if constexpr (KS > 1) {
+        if (!ks_tile(w, box_row0, bias, in)) break;
+      } else {
       // A k-slice of a tail tile writes its fp32 partial (this warp's 32 rows x
       // kTileN columns, column by column so each store is 128 contiguous bytes).
       float *part = nullptr;
@@ -1103,6 +1243,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
           if (lane == 0) atomicExch(counter, 0u);  // ready for the next call
         }
       }
+      }  // KS == 1
       if (NH == 1) {
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
@@ -1116,8 +1257,8 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
 
   tc_fence_before_sync();
   __syncwarp();
-  if constexpr (CG == 2)
-    cluster_sync_all();  // neither CTA leaves while its peer may still touch its shared memory
+  if constexpr (kCluster)
+    cluster_sync_all();  // no CTA leaves while a peer may still touch its shared memory
   else
     __syncthreads();
   tc_fence_after_sync();

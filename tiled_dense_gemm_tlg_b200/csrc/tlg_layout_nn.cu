@@ -3,7 +3,7 @@
 
 namespace tlg {
 
-const LayoutTables kLayoutNN = {TLG_LAYOUT(false, false), TLG_LAYOUT_PLAIN(false, false)};
+const LayoutTables kLayoutNN = {TLG_LAYOUT_NN, TLG_LAYOUT_PLAIN(false, false)};
 
 TLG_DEFINE_ERROR_WORD_READER(error_word_nn)
 

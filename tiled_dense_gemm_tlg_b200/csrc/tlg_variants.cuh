@@ -20,11 +20,13 @@ struct LaunchState {
   int units = 0;
 };
 
-template <int CG, int TN, int STAGES, bool OUT_F16, int EK, bool AT, bool BT, bool LSU>
+template <int CG, int TN, int STAGES, bool OUT_F16, int EK, bool AT, bool BT, bool LSU, int KS = 1>
 struct Variant {
   static constexpr int NH = TN > 256 ? 2 : 1;  // MMA halves per tile
   static constexpr int BN = TN / NH;           // the MMA's N
-  using Plan = SmemPlan<CG, BN, STAGES, NH>;
+  static constexpr int kClusterCtas = CG * KS;  // CTAs of one work unit (a cluster when > 1)
+  using Plan = SmemPlan<CG, BN, STAGES, NH, KS>;
+  static_assert(Plan::kDynamicBytes <= 232448, "shared memory per CTA exceeded");
 
   // attr must hold 2 entries.  With overlap_prev the kernel may start while
   // the previous kernel in the stream finishes (programmatic stream
@@ -41,9 +43,9 @@ struct Variant {
       attr[n].val.programmaticStreamSerializationAllowed = 1;
       ++n;
     }
-    if (CG == 2) {
+    if (kClusterCtas > 1) {
       attr[n].id = cudaLaunchAttributeClusterDimension;
-      attr[n].val.clusterDim.x = 2;
+      attr[n].val.clusterDim.x = kClusterCtas;
       attr[n].val.clusterDim.y = 1;
       attr[n].val.clusterDim.z = 1;
       ++n;
@@ -52,11 +54,11 @@ struct Variant {
     cfg->numAttrs = n;
   }
 
-  // Work units (CTAs, or CTA pairs) that can be resident at once: one per SM,
-  // or the number of 2-CTA clusters the occupancy calculator admits.
+  // Work units (CTAs, or clusters of CTAs) that can be resident at once: one per SM,
+  // or the number of clusters the occupancy calculator admits.
   static tlg_status units(int dev, int sms, int *out) {
     static LaunchState state[kMaxDevices];
-    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, EK, NH, AT, BT, LSU>;
+    auto kernel = gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, EK, NH, AT, BT, LSU, KS>;
     static std::mutex mutex;
     std::lock_guard<std::mutex> lock(mutex);
     LaunchState &st = state[dev];
@@ -67,11 +69,11 @@ struct Variant {
         return TLG_ERR_CUDA;
       }
       int n = sms;
-      if (CG == 2) {
+      if (kClusterCtas > 1) {
         cudaLaunchConfig_t cfg;
         cudaLaunchAttribute attr[2];
         fill_launch(&cfg, attr, nullptr);
-        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        cfg.gridDim = dim3(kClusterCtas * (sms / kClusterCtas), 1, 1);
         if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
           cudaGetLastError();
           return TLG_ERR_CUDA;
@@ -90,9 +92,9 @@ struct Variant {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[2];
     fill_launch(&cfg, attr, s, overlap_prev);
-    cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(units * kClusterCtas), 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, EK, NH, AT, BT, LSU>, tmA, tmB, tmC,
+        &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, EK, NH, AT, BT, LSU, KS>, tmA, tmB, tmC,
         p);
     if (e != cudaSuccess) {
       cudaGetLastError();
@@ -109,37 +111,46 @@ struct VariantFns {
 };
 
 
-constexpr int kNumVariants = 6;
+constexpr int kNumVariants = 9;
 
-#define TLG_FNS(CG, TN, ST, F16, BR, AT, BT, L)                  \
-  VariantFns {                                                   \
-    Variant<CG, TN, ST, F16, BR, AT, BT, L>::units,              \
-        Variant<CG, TN, ST, F16, BR, AT, BT, L>::launch          \
+#define TLG_FNS(CG, TN, ST, F16, BR, AT, BT, L, KS)                  \
+  VariantFns {                                                       \
+    Variant<CG, TN, ST, F16, BR, AT, BT, L, KS>::units,              \
+        Variant<CG, TN, ST, F16, BR, AT, BT, L, KS>::launch          \
   }
-#define TLG_VARIANT(CG, TN, ST, AT, BT, L)                                              \
+#define TLG_VARIANT_KS(CG, TN, ST, AT, BT, L, KS)                                       \
   {                                                                                     \
-    TLG_FNS(CG, TN, ST, false, kEpiNone, AT, BT, L),                                    \
-        TLG_FNS(CG, TN, ST, true, kEpiNone, AT, BT, L),                                 \
-        TLG_FNS(CG, TN, ST, true, kEpiFused, AT, BT, L),                                \
-        TLG_FNS(CG, TN, ST, false, kEpiFused, AT, BT, L),                               \
-        TLG_FNS(CG, TN, ST, true, kEpiBiasRelu, AT, BT, L)                              \
+    TLG_FNS(CG, TN, ST, false, kEpiNone, AT, BT, L, KS),                                \
+        TLG_FNS(CG, TN, ST, true, kEpiNone, AT, BT, L, KS),                             \
+        TLG_FNS(CG, TN, ST, true, kEpiFused, AT, BT, L, KS),                            \
+        TLG_FNS(CG, TN, ST, false, kEpiFused, AT, BT, L, KS),                           \
+        TLG_FNS(CG, TN, ST, true, kEpiBiasRelu, AT, BT, L, KS)                          \
   }
+#define TLG_VARIANT(CG, TN, ST, AT, BT, L) TLG_VARIANT_KS(CG, TN, ST, AT, BT, L, 1)
 #define TLG_NONE                                                                          \
   {                                                                                       \
     VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr}, \
         VariantFns{nullptr, nullptr}, VariantFns{nullptr, nullptr}                        \
   }
-#define TLG_LAYOUT(AT, BT)                                                                   \
-  {                                                                                          \
+// The TMA variants of one layout, in kBuilt's order.  The cluster k-split tiles
+// (the last three) are built for untransposed operands only (TLG_LAYOUT_NN).
+#define TLG_LAYOUT_COMMON(AT, BT)                                                            \
     TLG_VARIANT(1, 64, 8, AT, BT, false), TLG_VARIANT(1, 128, 6, AT, BT, false),             \
         TLG_VARIANT(1, 256, 4, AT, BT, false), TLG_VARIANT(2, 128, 8, AT, BT, false),        \
-        TLG_VARIANT(2, 256, 6, AT, BT, false), TLG_VARIANT(2, 512, 4, AT, BT, false)         \
+        TLG_VARIANT(2, 256, 6, AT, BT, false), TLG_VARIANT(2, 512, 4, AT, BT, false)
+#define TLG_LAYOUT(AT, BT) \
+  { TLG_LAYOUT_COMMON(AT, BT), TLG_NONE, TLG_NONE, TLG_NONE }
+#define TLG_LAYOUT_NN                                                                       \
+  {                                                                                         \
+    TLG_LAYOUT_COMMON(false, false), TLG_VARIANT_KS(1, 128, 5, false, false, false, 2),     \
+        TLG_VARIANT_KS(1, 256, 2, false, false, false, 2),                                  \
+        TLG_VARIANT_KS(1, 256, 2, false, false, false, 4)                                   \
   }
 // The same with plain loads, for the variants marked plain_loads in kBuilt.
 #define TLG_LAYOUT_PLAIN(AT, BT)                                                       \
   {                                                                                    \
     TLG_VARIANT(1, 64, 8, AT, BT, true), TLG_NONE, TLG_NONE, TLG_NONE,                 \
-        TLG_VARIANT(2, 256, 6, AT, BT, true), TLG_NONE                                 \
+        TLG_VARIANT(2, 256, 6, AT, BT, true), TLG_NONE, TLG_NONE, TLG_NONE, TLG_NONE   \
   }
 
 
