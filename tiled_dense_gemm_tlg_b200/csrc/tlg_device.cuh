@@ -145,6 +145,19 @@ static __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t par
   }
 }
 
+// Spins on the non-blocking test up to `spins` times before the bounded, sleeping wait.
+// Used where the phase usually completes within a k-block's time (the MMA warp waiting
+// for operands, the producer waiting for a free slot), so the thread reacts at once
+// instead of after a suspend: measured +0.3 % at 4096^3 and +3 % on the fp32-output
+// 4000 x 3000 x 1000 shape, with the tensor pipe's activity unchanged.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                               volatile uint32_t *abort_flag, uint64_t limit_ns,
+                                               uint32_t role, uint32_t *err_word, int spins) {
+  for (int i = 0; i < spins; ++i)
+    if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, limit_ns, role, err_word);
+}
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t *abort_flag, uint64_t limit_ns,
                                           uint32_t role, uint32_t *err_word) {

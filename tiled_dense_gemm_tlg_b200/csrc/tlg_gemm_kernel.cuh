@@ -661,8 +661,8 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       const int a_row = w.mb * kTileM + static_cast<int>(rank) * kBM;
       const int b_col = w.nb * kTileN + static_cast<int>(rank) * Plan::kBNc;
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
-        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
-                       &g_device_error)) {
+        if (!mbar_wait_spin(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
+                       &g_device_error, 4096)) {
           ok = false;
           break;
         }
@@ -796,8 +796,8 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
           }
           half1_ready();
         }
-        if (!mbar_wait(full_bar(stage), phase, abort_flag, p.limit_ns, kRoleMma,
-                       &g_device_error)) {
+        if (!mbar_wait_spin(full_bar(stage), phase, abort_flag, p.limit_ns, kRoleMma,
+                       &g_device_error, 4096)) {
           ok = false;
           break;
         }
