@@ -744,20 +744,25 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     // The MMAs of accumulator half h (h = 0 with NH == 1) for the k-block in ring slot st.
+    // Descriptors of ring slot 0; another slot, half or 16-k step only moves the start
+    // address, whose field (bits 0-13, in 16-byte units) never carries: shared-memory
+    // offsets stay below 256 KB.  K-major: 16 k = 32 bytes along the swizzled row;
+    // MN-major: 16 k = 16 rows of 128 bytes, 64-element blocks 8192 bytes apart.
+    const uint64_t adesc0 = !AT ? smem_desc_sw128(smem_u32(sA), 16, 1024)
+                                : smem_desc_sw128(smem_u32(sA), 8192, 1024);
+    const uint64_t bdesc0 = !BT ? smem_desc_sw128(smem_u32(sB), 8192, 1024)
+                                : smem_desc_sw128(smem_u32(sB), 16, 1024);
+    constexpr uint32_t kAStep = !AT ? 32 / 16 : 16 * 128 / 16;  // per 16 k, in 16-byte units
+    constexpr uint32_t kBStep = !BT ? 16 * 128 / 16 : 32 / 16;
     auto issue_half = [&](int st, int h, bool first_kb) {
-      const uint32_t a0 = smem_u32(sA + st * Plan::kABytes);
-      const uint32_t bh = smem_u32(sB + st * Plan::kBBytes) + h * Plan::kHalfBBytes;
+      const uint64_t ad = adesc0 + static_cast<uint32_t>(st * Plan::kABytes / 16);
+      const uint64_t bd =
+          bdesc0 + static_cast<uint32_t>((st * Plan::kBBytes + h * Plan::kHalfBBytes) / 16);
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((NH == 1 ? acc : h) * BN);
 #pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk) {
-        // K-major: 16 k = 32 bytes along the swizzled row; MN-major: 16 k
-        // = 16 rows of 128 bytes, 64-element blocks 8192 bytes apart.
-        const uint64_t adesc = !AT ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
-                                   : smem_desc_sw128(a0 + kk * 16 * 128, 8192, 1024);
-        const uint64_t bdesc = !BT ? smem_desc_sw128(bh + kk * 16 * 128, 8192, 1024)
-                                   : smem_desc_sw128(bh + kk * 32, 16, 1024);
-        mma_f16_ss<CG>(d_tmem, adesc, bdesc, idesc, (!first_kb || kk > 0) ? 1u : 0u);
-      }
+      for (int kk = 0; kk < kBK / 16; ++kk)
+        mma_f16_ss<CG>(d_tmem, ad + kk * kAStep, bd + kk * kBStep, idesc,
+                       (!first_kb || kk > 0) ? 1u : 0u);
     };
     for (int k = 0; k < n_work && ok; ++k) {
       const WorkItem w = item(k);
