@@ -64,7 +64,9 @@ static __device__ uint32_t g_device_error;
 // its own BN/CG columns of each half of B per k-block, plus two 4 KB output
 // boxes per epilogue warp.  With a cluster k-split (KS > 1 CTAs share one
 // tile's K range) each CTA also receives, for the BN/KS columns it finishes,
-// the fp32 partial sums of its KS - 1 peers.
+// the fp32 partial sums of its KS - 1 peers.  Where it still fits, the tile's
+// bias is kept there too, converted to fp32 once per tile (with two barriers
+// that pass it between the epilogue warps).
 template <int CG, int BN, int STAGES, int NH = 1, int KS = 1>
 struct SmemPlan {
   static constexpr int kBNc = BN / CG;  // B columns of one MMA half held by one CTA
@@ -78,9 +80,16 @@ struct SmemPlan {
   static constexpr uint32_t kRecvSlotBytes = kBM * kOwnCols * 4;  // one peer's fp32 partial of them
   static constexpr uint32_t kRecvOffset = kOutOffset + kOutBytes;
   static constexpr uint32_t kRecvBytes = (KS - 1) * kRecvSlotBytes;
-  static constexpr uint32_t kBarOffset = kRecvOffset + kRecvBytes;
+  static constexpr uint32_t kBiasOffset = kRecvOffset + kRecvBytes;
   // full, empty, tmem full/empty x2, drain; with a k-split also recv-full and send-free
-  static constexpr uint32_t kNumBars = 2 * STAGES + 4 + 1 + (KS > 1 ? 2 : 0);
+  static constexpr uint32_t kNumBarsBase = 2 * STAGES + 4 + 1 + (KS > 1 ? 2 : 0);
+  static constexpr uint32_t kBiasWant = BN * NH * 4;  // the tile's bias in fp32
+  static constexpr bool kBiasSmem =
+      kBiasOffset + kBiasWant + (kNumBarsBase + 2) * 8 + 16 + 1024 <= 232448;
+  static constexpr uint32_t kBiasBytes = kBiasSmem ? kBiasWant : 0;
+  static constexpr uint32_t kBarOffset = kBiasOffset + kBiasBytes;
+  // with the bias in shared memory also bias-full and bias-free
+  static constexpr uint32_t kNumBars = kNumBarsBase + (kBiasSmem ? 2 : 0);
   static constexpr uint32_t kMiscOffset = kBarOffset + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOffset + 16;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack to align the base to 1024
@@ -204,6 +213,52 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return r;
 }
 
+// Packed fp32 pairs.  sm_100's add/sub/mul/fma .f32x2 do two fp32 operations
+// in one instruction, each rounded exactly as its scalar form, so a pair of
+// columns costs the issue slot of one: the epilogue's arithmetic competes with
+// the producer and MMA warps for the SM's issue slots.  The pair sits in one
+// 64-bit register (the even column in the low word).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_splat(float c) { return f2_pack(c, c); }
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// x0 += b0, x1 += b1 as one packed add.
+__device__ __forceinline__ void f2_add_to(float &x0, float &x1, float b0, float b1) {
+  f2_unpack(f2_add(f2_pack(x0, x1), f2_pack(b0, b1)), x0, x1);
+}
+
 // GELU in its exact form x * Phi(x), Phi the standard normal CDF, in fp32.
 // Phi(-|x|) = erfc(z) / 2 with z = |x| / sqrt 2, and erfc is taken from
 // Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
@@ -225,6 +280,32 @@ __device__ __forceinline__ float gelu_erf(float x) {
   const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kH5, kH4), kH3), kH2), kH1);
   const float q = poly * ex2_approx(x * x * kE);  // Phi(-|x|)
   return x * (x < 0.0f ? q : 1.0f - q);
+}
+
+// gelu_erf on two values with the packed instructions: the same operations in
+// the same order, so the same bits.
+__device__ __forceinline__ void gelu_erf_2(float &x0, float &x1) {
+  constexpr float kPz = 0.3275911f * 0.70710678118654752f;
+  constexpr float kH1 = 0.5f * 0.254829592f, kH2 = 0.5f * -0.284496736f,
+                  kH3 = 0.5f * 1.421413741f, kH4 = 0.5f * -1.453152027f,
+                  kH5 = 0.5f * 1.061405429f;
+  constexpr float kE = -0.5f * 1.4426950408889634f;
+  const uint64_t x = f2_pack(x0, x1);
+  const uint64_t t = f2_pack(rcp_approx(fmaf(kPz, fabsf(x0), 1.0f)),
+                             rcp_approx(fmaf(kPz, fabsf(x1), 1.0f)));
+  uint64_t poly = f2_fma(t, f2_splat(kH5), f2_splat(kH4));
+  poly = f2_fma(t, poly, f2_splat(kH3));
+  poly = f2_fma(t, poly, f2_splat(kH2));
+  poly = f2_fma(t, poly, f2_splat(kH1));
+  poly = f2_mul(t, poly);
+  float z0, z1;
+  f2_unpack(f2_mul(f2_mul(x, x), f2_splat(kE)), z0, z1);
+  const uint64_t q = f2_mul(poly, f2_pack(ex2_approx(z0), ex2_approx(z1)));  // Phi(-|x|)
+  const uint64_t omq = f2_sub(f2_splat(1.0f), q);
+  float q0, q1, o0, o1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(omq, o0, o1);
+  f2_unpack(f2_mul(x, f2_pack(x0 < 0.0f ? q0 : o0, x1 < 0.0f ? q1 : o1)), x0, x1);
 }
 
 // SiLU and the tanh form of GELU are both x * sigmoid(c1 x + c3 x^3):
@@ -249,6 +330,16 @@ __device__ __forceinline__ float sigmoid_form_apply(SigmoidForm f, float x) {
   return x * rcp_approx(1.0f + ex2_approx(z));
 }
 
+// sigmoid_form_apply on two values with the packed instructions (same bits).
+__device__ __forceinline__ void sigmoid_form_apply_2(SigmoidForm f, float &x0, float &x1) {
+  const uint64_t x = f2_pack(x0, x1);
+  float z0, z1;
+  f2_unpack(f2_mul(x, f2_fma(f2_splat(f.c3), f2_mul(x, x), f2_splat(f.c1))), z0, z1);
+  float d0, d1;
+  f2_unpack(f2_add(f2_splat(1.0f), f2_pack(ex2_approx(z0), ex2_approx(z1))), d0, d1);
+  f2_unpack(f2_mul(x, f2_pack(rcp_approx(d0), rcp_approx(d1))), x0, x1);
+}
+
 __device__ __forceinline__ float activate(int act, float x) {
   if (act == kActRelu) return fmaxf(x, 0.0f);
   if (act == kActGelu) return gelu_erf(x);
@@ -264,11 +355,11 @@ __device__ __forceinline__ void activate_32(int act, float (&v)[32]) {
     for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
   } else if (act == kActGelu) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+    for (int j = 0; j < 32; j += 2) gelu_erf_2(v[j], v[j + 1]);
   } else if (act == kActSilu || act == kActGeluTanh) {
     const SigmoidForm f = sigmoid_form(act);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = sigmoid_form_apply(f, v[j]);
+    for (int j = 0; j < 32; j += 2) sigmoid_form_apply_2(f, v[j], v[j + 1]);
   }
 }
 
@@ -292,8 +383,7 @@ __device__ __forceinline__ void add_residual_32(const GemmParams &p, int row, in
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __half22float2(h[e]);
-          v[c * 8 + 2 * e] += f.x;
-          v[c * 8 + 2 * e + 1] += f.y;
+          f2_add_to(v[c * 8 + 2 * e], v[c * 8 + 2 * e + 1], f.x, f.y);
         }
       }
     } else {
@@ -308,10 +398,8 @@ __device__ __forceinline__ void add_residual_32(const GemmParams &p, int row, in
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const float4 w = q[c];
-        v[4 * c] += w.x;
-        v[4 * c + 1] += w.y;
-        v[4 * c + 2] += w.z;
-        v[4 * c + 3] += w.w;
+        f2_add_to(v[4 * c], v[4 * c + 1], w.x, w.y);
+        f2_add_to(v[4 * c + 2], v[4 * c + 3], w.z, w.w);
       }
     } else {
 #pragma unroll
@@ -403,8 +491,19 @@ __device__ __forceinline__ void add_bias_slice_32(const BiasSlice<CPL> &s, int t
     // columns t0 + 2jj and t0 + 2jj + 1 sit in one word of lane (t0 + 2jj) / CPL
     const uint32_t w = __shfl_sync(0xffffffffu, s.w[((2 * jj) % CPL) / 2], (t0 + 2 * jj) / CPL);
     const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
-    v[2 * jj] += f.x;
-    v[2 * jj + 1] += f.y;
+    f2_add_to(v[2 * jj], v[2 * jj + 1], f.x, f.y);
+  }
+}
+
+// v[j] += bias[tile column t0 + j], j < 32, from the tile's fp32 bias in
+// shared memory at sbias: every lane reads the same 16 bytes at a time (a
+// broadcast), two packed adds each.
+__device__ __forceinline__ void add_bias_smem_32(uint32_t sbias, int t0, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint4 b = ld_shared_v4(sbias + static_cast<uint32_t>(t0 + 4 * q) * 4u);
+    f2_add_to(v[4 * q], v[4 * q + 1], __uint_as_float(b.x), __uint_as_float(b.y));
+    f2_add_to(v[4 * q + 2], v[4 * q + 3], __uint_as_float(b.z), __uint_as_float(b.w));
   }
 }
 
@@ -412,12 +511,17 @@ __device__ __forceinline__ void add_bias_slice_32(const BiasSlice<CPL> &s, int t
 // 64-column piece at tile column tcol: + bias, activation, + residual.  Done
 // one half at a time so that the first half is packed for the store (and its
 // registers freed) before the second half's activation runs.
-template <bool OUT_F16, bool ON, int CPL>
+template <bool OUT_F16, bool ON, bool SBIAS, int CPL>
 __device__ __forceinline__ void epi_apply_32(const GemmParams &p, const EpiIn<ON> &in,
-                                             const BiasSlice<CPL> &bias, int row, int col0,
-                                             int tcol, int half, float (&v)[32]) {
+                                             const BiasSlice<CPL> &bias, uint32_t sbias, int row,
+                                             int col0, int tcol, int half, float (&v)[32]) {
   const int c0 = col0 + 32 * half;
-  if (p.bias != nullptr) add_bias_slice_32<CPL>(bias, tcol + 32 * half, v);
+  if (p.bias != nullptr) {
+    if constexpr (SBIAS)
+      add_bias_smem_32(sbias, tcol + 32 * half, v);
+    else
+      add_bias_slice_32<CPL>(bias, tcol + 32 * half, v);
+  }
   activate_32(p.act, v);
   if (p.R != nullptr) {
     if (ON && in.has_r) {
@@ -427,8 +531,7 @@ __device__ __forceinline__ void epi_apply_32(const GemmParams &p, const EpiIn<ON
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __half22float2(h[e]);
-          v[c * 8 + 2 * e] += f.x;
-          v[c * 8 + 2 * e + 1] += f.y;
+          f2_add_to(v[c * 8 + 2 * e], v[c * 8 + 2 * e + 1], f.x, f.y);
         }
       }
     } else {
@@ -440,6 +543,15 @@ __device__ __forceinline__ void epi_apply_32(const GemmParams &p, const EpiIn<ON
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// pack_half2 followed by max(., 0) on both halves.  Rounding is monotonic and
+// 0 is exact, so this equals rounding max(x, 0); like fmaxf, max.f16x2 returns
+// the other operand for a NaN, so ReLU(NaN) = 0 as in the fp32 form.
+__device__ __forceinline__ uint32_t pack_half2_relu(float lo, float hi) {
+  uint32_t r;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(pack_half2(lo, hi)), "r"(0u));
+  return r;
 }
 
 // Writes one 128-byte row piece (eight 16-byte pieces) of a 32-row output box
@@ -582,6 +694,10 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
   // peer has consumed this CTA's partials from its own receive buffer.
   const uint32_t recv_full_bar = bar0 + 8u * (2 * STAGES + 5);
   const uint32_t send_free_bar = bar0 + 8u * (2 * STAGES + 6);
+  // Bias in shared memory: every epilogue warp has written its share of the tile's
+  // bias / has done reading it.
+  const uint32_t bias_full_bar = bar0 + 8u * Plan::kNumBarsBase;
+  const uint32_t bias_free_bar = bar0 + 8u * (Plan::kNumBarsBase + 1);
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + Plan::kMiscOffset);
   uint32_t *tmem_holder = misc;
   volatile uint32_t *abort_flag = misc + 1;
@@ -623,6 +739,10 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     if constexpr (KS > 1) {
       mbar_init(recv_full_bar, (KS - 1) * 32 * kEpiWarps);  // every epilogue thread of each peer
       mbar_init(send_free_bar, (KS - 1) * 32 * kEpiWarps);
+    }
+    if constexpr (Plan::kBiasSmem) {
+      mbar_init(bias_full_bar, kEpiWarps);  // lane 0 of each epilogue warp
+      mbar_init(bias_free_bar, kEpiWarps);
     }
     *abort_flag = 0u;
     fence_mbar_init();
@@ -956,16 +1076,29 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     // their latency passes while this piece is stored.
     constexpr int kCPL = kTileN / 32;  // bias columns per lane
     constexpr bool kPrefR = EK == kEpiFused && OUT_F16 && !LSU;  // residual pieces loaded ahead
+    // The tile's bias in fp32 in shared memory (where the plan has room for it), else
+    // spread over the lanes as fp16 and fetched by shuffles.
+    constexpr bool kSBias = EK != kEpiNone && Plan::kBiasSmem;
+    const uint32_t sbias = smem_u32(smem + Plan::kBiasOffset);
     // The epilogue of one 32-column half of a piece (tile columns tcol + 32*half ..).
+    // bias + ReLU (fp16 C only) leaves the ReLU to the packing.
+    static_assert(EK != kEpiBiasRelu || OUT_F16, "the bias + ReLU build writes fp16");
     auto epi32 = [&](const EpiIn<kPrefR> &in, const BiasSlice<kCPL> &bias, int row, int col0,
                      int tcol, int half, float(&v)[32]) {
       if constexpr (EK == kEpiFused) {
-        epi_apply_32<OUT_F16, kPrefR, kCPL>(p, in, bias, row, col0, tcol, half, v);
+        epi_apply_32<OUT_F16, kPrefR, kSBias, kCPL>(p, in, bias, sbias, row, col0, tcol, half, v);
       } else if constexpr (EK == kEpiBiasRelu) {
-        add_bias_slice_32<kCPL>(bias, tcol + 32 * half, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
+        if constexpr (kSBias)
+          add_bias_smem_32(sbias, tcol + 32 * half, v);
+        else
+          add_bias_slice_32<kCPL>(bias, tcol + 32 * half, v);
       }
+    };
+    auto pack = [&](float lo, float hi) {
+      if constexpr (EK == kEpiBiasRelu)
+        return pack_half2_relu(lo, hi);
+      else
+        return pack_half2(lo, hi);
     };
     auto emit64 = [&](float (&va)[32], float (&vb)[32], int box_row0, int col0, int tcol,
                       const BiasSlice<kCPL> &bias, EpiIn<kPrefR> &in, int next_col0) {
@@ -973,10 +1106,10 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         uint32_t h[32];  // 64 fp16 values, round to nearest even
         epi32(in, bias, box_row0 + lane, col0, tcol, 0, va);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) h[j] = pack_half2(va[2 * j], va[2 * j + 1]);
+        for (int j = 0; j < 16; ++j) h[j] = pack(va[2 * j], va[2 * j + 1]);
         epi32(in, bias, box_row0 + lane, col0, tcol, 1, vb);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) h[16 + j] = pack_half2(vb[2 * j], vb[2 * j + 1]);
+        for (int j = 0; j < 16; ++j) h[16 + j] = pack(vb[2 * j], vb[2 * j + 1]);
         if constexpr (kPrefR) {
           if (next_col0 >= 0) epi_prefetch<kPrefR>(p, box_row0 + lane, next_col0, in);
         }
@@ -1131,7 +1264,25 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       // loop still runs.
       EpiIn<kPrefR> in;
       BiasSlice<kCPL> bias;
-      if constexpr (EK != kEpiNone) {
+      if constexpr (kSBias) {
+        if (p.bias != nullptr) {
+          // The shared bias buffer holds one tile's bias: once every epilogue warp is
+          // done with the previous tile's, each writes its share of this tile's.
+          if (k > 0 && !mbar_wait(bias_free_bar, (k - 1) & 1, abort_flag, p.limit_ns,
+                                  kRoleEpilogue, &g_device_error))
+            break;
+          float *sb = reinterpret_cast<float *>(smem + Plan::kBiasOffset);
+          for (int c = (warp - 2) * 32 + lane; c < kTileN; c += 32 * kEpiWarps) {
+            const int col = w.nb * kTileN + c;
+            sb[c] = col < p.N ? __half2float(p.bias[col]) : 0.0f;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bias_full_bar);
+          if (!mbar_wait(bias_full_bar, k & 1, abort_flag, p.limit_ns, kRoleEpilogue,
+                         &g_device_error))
+            break;
+        }
+      } else if constexpr (EK != kEpiNone) {
         if (p.bias != nullptr && w.nb * kTileN < p.N) load_bias_slice<kCPL>(p, w.nb * kTileN, lane, bias);
       }
       if constexpr (kPrefR) {
@@ -1249,6 +1400,12 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         }
       }
       }  // KS == 1
+      if constexpr (kSBias) {
+        if (p.bias != nullptr) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bias_free_bar);  // this warp is done with the tile's bias
+        }
+      }
       if (NH == 1) {
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
