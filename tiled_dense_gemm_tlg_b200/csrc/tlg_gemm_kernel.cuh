@@ -213,7 +213,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return r;
 }
 
-// Packed fp32 pairs.  sm_100's add/sub/mul/fma .f32x2 do two fp32 operations
+// Packed fp32 pairs.  sm_100's add/mul/fma .f32x2 do two fp32 operations
 // in one instruction, each rounded exactly as its scalar form, so a pair of
 // columns costs the issue slot of one: the epilogue's arithmetic competes with
 // the producer and MMA warps for the SM's issue slots.  The pair sits in one
@@ -236,12 +236,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return r;
 }
 
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -259,6 +253,16 @@ __device__ __forceinline__ void f2_add_to(float &x0, float &x1, float b0, float 
   f2_unpack(f2_add(f2_pack(x0, x1), f2_pack(b0, b1)), x0, x1);
 }
 
+// x0 += the low fp16 half of w, x1 += its high half: sm_100's mixed-precision
+// add takes the fp16 operand as it is (no conversion instruction) and rounds
+// the fp32 sum once, exactly as a conversion followed by an fp32 add.
+__device__ __forceinline__ void add_half2_to(float &x0, float &x1, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %1, hi, %1;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "r"(w));
+}
+
 // GELU in its exact form x * Phi(x), Phi the standard normal CDF, in fp32.
 // Phi(-|x|) = erfc(z) / 2 with z = |x| / sqrt 2, and erfc is taken from
 // Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
@@ -266,10 +270,13 @@ __device__ __forceinline__ void f2_add_to(float &x0, float &x1, float b0, float 
 //   erfc(z) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),
 //   t = 1 / (1 + p z).
 // Here 1/sqrt 2 is folded into p, the 1/2 into the a_i, and exp(-z^2) =
-// 2^(x^2 * (-log2(e) / 2)).  That gives Phi(-|x|) directly (no cancellation
-// in the negative tail) and Phi(|x|) = 1 - Phi(-|x|).  Branch-free, so the 32
-// values a thread holds are evaluated side by side; every instruction counts,
-// since the epilogue's arithmetic competes with the tensor pipe for the SM.
+// 2^(x^2 * (-log2(e) / 2)).  That gives q = Phi(-|x|) directly (no
+// cancellation in the negative tail), and since Phi(|x|) = 1 - q,
+//   x Phi(x) = max(x, 0) - |x| q
+// (x (1 - q) for x >= 0, -|x| q for x < 0): one fused multiply-add, no
+// select.  Branch-free, so the 32 values a thread holds are evaluated side by
+// side; every instruction counts, since the epilogue's arithmetic competes
+// with the tensor pipe for the SM.
 __device__ __forceinline__ float gelu_erf(float x) {
   constexpr float kPz = 0.3275911f * 0.70710678118654752f;
   constexpr float kH1 = 0.5f * 0.254829592f, kH2 = 0.5f * -0.284496736f,
@@ -279,7 +286,7 @@ __device__ __forceinline__ float gelu_erf(float x) {
   const float t = rcp_approx(fmaf(kPz, fabsf(x), 1.0f));
   const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kH5, kH4), kH3), kH2), kH1);
   const float q = poly * ex2_approx(x * x * kE);  // Phi(-|x|)
-  return x * (x < 0.0f ? q : 1.0f - q);
+  return fmaf(-fabsf(x), q, fmaxf(x, 0.0f));
 }
 
 // gelu_erf on two values with the packed instructions: the same operations in
@@ -300,12 +307,10 @@ __device__ __forceinline__ void gelu_erf_2(float &x0, float &x1) {
   poly = f2_mul(t, poly);
   float z0, z1;
   f2_unpack(f2_mul(f2_mul(x, x), f2_splat(kE)), z0, z1);
-  const uint64_t q = f2_mul(poly, f2_pack(ex2_approx(z0), ex2_approx(z1)));  // Phi(-|x|)
-  const uint64_t omq = f2_sub(f2_splat(1.0f), q);
-  float q0, q1, o0, o1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(omq, o0, o1);
-  f2_unpack(f2_mul(x, f2_pack(x0 < 0.0f ? q0 : o0, x1 < 0.0f ? q1 : o1)), x0, x1);
+  float q0, q1;  // Phi(-|x|)
+  f2_unpack(f2_mul(poly, f2_pack(ex2_approx(z0), ex2_approx(z1))), q0, q1);
+  x0 = fmaf(-fabsf(x0), q0, fmaxf(x0, 0.0f));
+  x1 = fmaf(-fabsf(x1), q1, fmaxf(x1, 0.0f));
 }
 
 // SiLU and the tanh form of GELU are both x * sigmoid(c1 x + c3 x^3):
@@ -379,12 +384,10 @@ __device__ __forceinline__ void add_residual_32(const GemmParams &p, int row, in
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const uint4 w = q[c];
-        const __half2 *h = reinterpret_cast<const __half2 *>(&w);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(h[e]);
-          f2_add_to(v[c * 8 + 2 * e], v[c * 8 + 2 * e + 1], f.x, f.y);
-        }
+        add_half2_to(v[c * 8], v[c * 8 + 1], w.x);
+        add_half2_to(v[c * 8 + 2], v[c * 8 + 3], w.y);
+        add_half2_to(v[c * 8 + 4], v[c * 8 + 5], w.z);
+        add_half2_to(v[c * 8 + 6], v[c * 8 + 7], w.w);
       }
     } else {
 #pragma unroll
@@ -490,8 +493,7 @@ __device__ __forceinline__ void add_bias_slice_32(const BiasSlice<CPL> &s, int t
   for (int jj = 0; jj < 16; ++jj) {
     // columns t0 + 2jj and t0 + 2jj + 1 sit in one word of lane (t0 + 2jj) / CPL
     const uint32_t w = __shfl_sync(0xffffffffu, s.w[((2 * jj) % CPL) / 2], (t0 + 2 * jj) / CPL);
-    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
-    f2_add_to(v[2 * jj], v[2 * jj + 1], f.x, f.y);
+    add_half2_to(v[2 * jj], v[2 * jj + 1], w);
   }
 }
 
@@ -527,12 +529,11 @@ __device__ __forceinline__ void epi_apply_32(const GemmParams &p, const EpiIn<ON
     if (ON && in.has_r) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const __half2 *h = reinterpret_cast<const __half2 *>(&in.r[4 * half + c]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(h[e]);
-          f2_add_to(v[c * 8 + 2 * e], v[c * 8 + 2 * e + 1], f.x, f.y);
-        }
+        const uint4 w = in.r[4 * half + c];
+        add_half2_to(v[c * 8], v[c * 8 + 1], w.x);
+        add_half2_to(v[c * 8 + 2], v[c * 8 + 3], w.y);
+        add_half2_to(v[c * 8 + 4], v[c * 8 + 5], w.z);
+        add_half2_to(v[c * 8 + 6], v[c * 8 + 7], w.w);
       }
     } else {
       add_residual_32<OUT_F16>(p, row, c0, v);
