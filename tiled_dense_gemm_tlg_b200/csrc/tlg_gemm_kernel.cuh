@@ -264,53 +264,53 @@ __device__ __forceinline__ void add_half2_to(float &x0, float &x1, uint32_t w) {
 }
 
 // GELU in its exact form x * Phi(x), Phi the standard normal CDF, in fp32.
-// Phi(-|x|) = erfc(z) / 2 with z = |x| / sqrt 2, and erfc is taken from
-// Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
-// (Hastings' rational approximation, |error| <= 1.5e-7 for z >= 0):
-//   erfc(z) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),
-//   t = 1 / (1 + p z).
-// Here 1/sqrt 2 is folded into p, the 1/2 into the a_i, and exp(-z^2) =
-// 2^(x^2 * (-log2(e) / 2)).  That gives q = Phi(-|x|) directly (no
-// cancellation in the negative tail), and since Phi(|x|) = 1 - q,
-//   x Phi(x) = max(x, 0) - |x| q
-// (x (1 - q) for x >= 0, -|x| q for x < 0): one fused multiply-add, no
-// select.  Branch-free, so the 32 values a thread holds are evaluated side by
-// side; every instruction counts, since the epilogue's arithmetic competes
-// with the tensor pipe for the SM.
-__device__ __forceinline__ float gelu_erf(float x) {
-  constexpr float kPz = 0.3275911f * 0.70710678118654752f;
-  constexpr float kH1 = 0.5f * 0.254829592f, kH2 = 0.5f * -0.284496736f,
-                  kH3 = 0.5f * 1.421413741f, kH4 = 0.5f * -1.453152027f,
-                  kH5 = 0.5f * 1.061405429f;
-  constexpr float kE = -0.5f * 1.4426950408889634f;
-  const float t = rcp_approx(fmaf(kPz, fabsf(x), 1.0f));
-  const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kH5, kH4), kH3), kH2), kH1);
-  const float q = poly * ex2_approx(x * x * kE);  // Phi(-|x|)
-  return fmaf(-fabsf(x), q, fmaxf(x, 0.0f));
+// With a = min(|x|, 6) and q = Phi(-a), the standard normal tail,
+//   x Phi(x) = max(x, 0) - a q
+// (x (1 - q) for x >= 0, -|x| q for x < 0; beyond |x| = 6, q < 1e-9 and a q
+// < 6e-9): one fused multiply-add, no select, and q is computed directly, so
+// the negative tail has no cancellation.  q = 2^g(a) with g a degree-6
+// polynomial fitted to log2 Phi(-a) on [0, 6], its error weighted by what it
+// costs in GELU (a Phi(-a) ln 2) and made near-minimax by Lawson's
+// reweighted least squares (fit_gelu_tail.py beside this file prints the
+// coefficients; GELU error below 3e-7 on [-8, 8] in fp32).  One exp2 and no
+// reciprocal: the special-function unit the epilogue shares with its SM
+// partition is its scarcest resource.  min.NaN keeps a NaN input NaN.
+constexpr float kGeluG0 = -0.999993086f, kGeluG1 = -1.15120173f, kGeluG2 = -0.458770931f,
+                kGeluG3 = -0.0534121692f, kGeluG4 = 0.00808076002f, kGeluG5 = -0.000769232807f,
+                kGeluG6 = 3.30943076e-05f;
+
+__device__ __forceinline__ float gelu_tail_arg(float x) {  // min(|x|, 6), NaN stays NaN
+  float a;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(a) : "f"(fabsf(x)), "f"(6.0f));
+  return a;
 }
 
-// gelu_erf on two values with the packed instructions: the same operations in
-// the same order, so the same bits.
+__device__ __forceinline__ float gelu_erf(float x) {
+  const float a = gelu_tail_arg(x);
+  float g = fmaf(kGeluG6, a, kGeluG5);
+  g = fmaf(g, a, kGeluG4);
+  g = fmaf(g, a, kGeluG3);
+  g = fmaf(g, a, kGeluG2);
+  g = fmaf(g, a, kGeluG1);
+  g = fmaf(g, a, kGeluG0);
+  return fmaf(-a, ex2_approx(g), fmaxf(x, 0.0f));  // q = 2^g = Phi(-a)
+}
+
+// gelu_erf on two values, the polynomial with the packed instructions: the same
+// operations in the same order, so the same bits.
 __device__ __forceinline__ void gelu_erf_2(float &x0, float &x1) {
-  constexpr float kPz = 0.3275911f * 0.70710678118654752f;
-  constexpr float kH1 = 0.5f * 0.254829592f, kH2 = 0.5f * -0.284496736f,
-                  kH3 = 0.5f * 1.421413741f, kH4 = 0.5f * -1.453152027f,
-                  kH5 = 0.5f * 1.061405429f;
-  constexpr float kE = -0.5f * 1.4426950408889634f;
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t t = f2_pack(rcp_approx(fmaf(kPz, fabsf(x0), 1.0f)),
-                             rcp_approx(fmaf(kPz, fabsf(x1), 1.0f)));
-  uint64_t poly = f2_fma(t, f2_splat(kH5), f2_splat(kH4));
-  poly = f2_fma(t, poly, f2_splat(kH3));
-  poly = f2_fma(t, poly, f2_splat(kH2));
-  poly = f2_fma(t, poly, f2_splat(kH1));
-  poly = f2_mul(t, poly);
-  float z0, z1;
-  f2_unpack(f2_mul(f2_mul(x, x), f2_splat(kE)), z0, z1);
-  float q0, q1;  // Phi(-|x|)
-  f2_unpack(f2_mul(poly, f2_pack(ex2_approx(z0), ex2_approx(z1))), q0, q1);
-  x0 = fmaf(-fabsf(x0), q0, fmaxf(x0, 0.0f));
-  x1 = fmaf(-fabsf(x1), q1, fmaxf(x1, 0.0f));
+  const float a0 = gelu_tail_arg(x0), a1 = gelu_tail_arg(x1);
+  const uint64_t a = f2_pack(a0, a1);
+  uint64_t g = f2_fma(f2_splat(kGeluG6), a, f2_splat(kGeluG5));
+  g = f2_fma(g, a, f2_splat(kGeluG4));
+  g = f2_fma(g, a, f2_splat(kGeluG3));
+  g = f2_fma(g, a, f2_splat(kGeluG2));
+  g = f2_fma(g, a, f2_splat(kGeluG1));
+  g = f2_fma(g, a, f2_splat(kGeluG0));
+  float g0, g1;
+  f2_unpack(g, g0, g1);
+  x0 = fmaf(-a0, ex2_approx(g0), fmaxf(x0, 0.0f));
+  x1 = fmaf(-a1, ex2_approx(g1), fmaxf(x1, 0.0f));
 }
 
 // SiLU and the tanh form of GELU are both x * sigmoid(c1 x + c3 x^3):
