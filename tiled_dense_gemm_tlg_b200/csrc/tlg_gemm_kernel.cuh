@@ -727,6 +727,15 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     return w;
   };
 
+  // The k-blocks of a unit's item k in processing order: whole tiles walk K
+  // ascending on even k and descending on odd k, so a tile starts on the k-blocks
+  // the unit's previous tile (and its wave's) read last, which L2 still holds.
+  // Tail slices, k-split slices and the plain-load path keep ascending order.
+  auto kb_at = [&](const WorkItem &w, int k, int i) {
+    const bool down = !LSU && KS == 1 && w.tail < 0 && (k & 1) != 0;
+    return down ? w.kb1 - 1 - i : w.kb0 + i;
+  };
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), LSU ? kLoaderWarps * CG : 1);
@@ -781,7 +790,8 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       const WorkItem w = item(k);
       const int a_row = w.mb * kTileM + static_cast<int>(rank) * kBM;
       const int b_col = w.nb * kTileN + static_cast<int>(rank) * Plan::kBNc;
-      for (int kb = w.kb0; kb < w.kb1; ++kb) {
+      for (int i = 0; i < w.kb1 - w.kb0; ++i) {
+        const int kb = kb_at(w, k, i);
         if (!mbar_wait_spin(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
                        &g_device_error, 4096)) {
           ok = false;
@@ -912,7 +922,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         }
         pend = 0;
       };
-      for (int kb = w.kb0; kb < w.kb1; ++kb) {
+      for (int i = 0; i < w.kb1 - w.kb0; ++i) {
         if (NH == 2 && !half1_free && pend == STAGES) {
           // every slot holds a run-ahead k-block: nothing more can land before half 1 is free
           if (!mbar_wait(tempty_bar(1), acc_phase ^ 1u, abort_flag, p.limit_ns, kRoleMma,
@@ -931,11 +941,11 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         if (NH == 2 && !half1_free && mbar_test_wait(tempty_bar(1), acc_phase ^ 1u)) half1_ready();
         if (NH == 2 && !half1_free) {
           if (pend == 0) pend_stage = stage;
-          issue_half(stage, 0, kb == w.kb0);
+          issue_half(stage, 0, i == 0);
           ++pend;
         } else {
 #pragma unroll
-          for (int h = 0; h < NH; ++h) issue_half(stage, h, kb == w.kb0);
+          for (int h = 0; h < NH; ++h) issue_half(stage, h, i == 0);
           mma_commit<CG>(empty_bar(stage));
         }
         if (++stage == STAGES) {
