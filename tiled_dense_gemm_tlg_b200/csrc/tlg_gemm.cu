@@ -860,7 +860,7 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   // stored transposed; B 64 n x 64 k, or 64 k x (columns per CTA) when stored
   // transposed; C 128 bytes x 32 rows.
   // (Maps a path does not use stay zeroed and are never read by the kernel.)
-  CUtensorMap tmA = {}, tmB = {}, tmC = {};
+  CUtensorMap tmA = {}, tmB = {}, tmC = {}, tmR = {};
   const CUtensorMapDataType h16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const CUtensorMapDataType c_type = f16 ? h16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const uint32_t b_rows_per_cta =
@@ -903,10 +903,17 @@ tlg_status gemm_impl(int64_t M, int64_t N, int64_t K, bool at, const void *A, in
   p.R = e.R;
   p.ldr = e.ldr;
   p.r_vec = (e.R != nullptr && aligned16(e.R) && (e.ldr * osz) % 16 == 0) ? 1 : 0;
+  // An fp16 residual TMA can describe: the last tile of each unit stages it in the ring
+  // (32 x 64 boxes, the epilogue warps' pieces).
+  p.r_tma = 0;
+  if (ek == kEpiFused && f16 && !plain && p.r_vec != 0 &&
+      encode_2d(&tmR, h16, e.R, uint64_t(N), uint64_t(M), uint64_t(e.ldr) * 2, 64, 32))
+    p.r_tma = 1;
   // After this call's own copy kernel the GEMM starts as its programmatic
   // dependent: its set-up overlaps the copy's tail.
   const tlg_status ls = fns_for(rv.idx, f16, ek, at, bt, plain)
-                             .launch(rv.sched.units, tmA, tmB, tmC, p, rv.cfg.overlap_prev != 0 || copy_ab, s);
+                             .launch(rv.sched.units, tmA, tmB, tmC, tmR, p,
+                                     rv.cfg.overlap_prev != 0 || copy_ab, s);
   if (ls != TLG_OK || !copy_c) return ls;
   const CopyJob jc = {static_cast<const char *>(C_use), aligned_ld(N, osz) * osz, static_cast<char *>(C),
                       ldc * osz, M, N * osz};

@@ -85,11 +85,11 @@ struct SmemPlan {
   static constexpr uint32_t kNumBarsBase = 2 * STAGES + 4 + 1 + (KS > 1 ? 2 : 0);
   static constexpr uint32_t kBiasWant = BN * NH * 4;  // the tile's bias in fp32
   static constexpr bool kBiasSmem =
-      kBiasOffset + kBiasWant + (kNumBarsBase + 2) * 8 + 16 + 1024 <= 232448;
+      kBiasOffset + kBiasWant + (kNumBarsBase + 3) * 8 + 16 + 1024 <= 232448;
   static constexpr uint32_t kBiasBytes = kBiasSmem ? kBiasWant : 0;
   static constexpr uint32_t kBarOffset = kBiasOffset + kBiasBytes;
-  // with the bias in shared memory also bias-full and bias-free
-  static constexpr uint32_t kNumBars = kNumBarsBase + (kBiasSmem ? 2 : 0);
+  // with the bias in shared memory also bias-full and bias-free; last, residual-full
+  static constexpr uint32_t kNumBars = kNumBarsBase + (kBiasSmem ? 2 : 0) + 1;
   static constexpr uint32_t kMiscOffset = kBarOffset + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOffset + 16;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack to align the base to 1024
@@ -127,6 +127,7 @@ struct GemmParams {
   const void *R;     // residual in C's type, or nullptr; may be C itself (same ldc)
   int64_t ldr;
   int r_vec;         // R's base and row stride are 16-byte aligned
+  int r_tma;         // tmR describes R (fp16 C, TMA path): the last tile's residual is staged
 };
 
 // One unit of work: a tile, or one k-slice of a tail tile.
@@ -669,7 +670,8 @@ template <int CG, int BN, int STAGES, bool OUT_F16, int EK, int NH = 1, bool AT 
 __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmC,
+                      const __grid_constant__ CUtensorMap tmR, const GemmParams p) {
   using Plan = SmemPlan<CG, BN, STAGES, NH, KS>;
   constexpr int kTileM = kBM * CG;
   constexpr int kTileN = BN * NH;
@@ -699,6 +701,25 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
   // bias / has done reading it.
   const uint32_t bias_full_bar = bar0 + 8u * Plan::kNumBarsBase;
   const uint32_t bias_free_bar = bar0 + 8u * (Plan::kNumBarsBase + 1);
+  // The last item's residual boxes have landed in the ring (see the producer).
+  const uint32_t res_bar = bar0 + 8u * (Plan::kNumBars - 1);
+  // Staging of the last tile's fp16 residual (fused epilogue, TMA path, whole tiles of one
+  // accumulator): kResBoxes boxes of 32 rows x 64 columns (4 KB, 128-byte swizzle), box
+  // j = quarter * kResPieces + piece, kResPerStage to a ring slot (its A part, then its B
+  // part), starting at the first slot the producer would fill next.
+  constexpr bool kResSmem = EK == kEpiFused && OUT_F16 && KS == 1 && NH == 1 && !LSU;
+  constexpr int kResPieces = kTileN / 64;
+  constexpr int kResBoxes = (kBM / 32) * kResPieces;
+  constexpr int kResPerA = static_cast<int>(Plan::kABytes / 4096);
+  constexpr int kResPerStage = kResPerA + static_cast<int>(Plan::kBBytes / 4096);
+  constexpr int kResStages = (kResBoxes + kResPerStage - 1) / kResPerStage;
+  static_assert(!kResSmem || kResStages <= STAGES, "the residual of a tile fits the ring");
+  auto res_box = [&](int first_stage, int j) -> uint32_t {
+    const int st = (first_stage + j / kResPerStage) % STAGES;
+    const int b = j % kResPerStage;
+    return b < kResPerA ? smem_u32(sA + st * Plan::kABytes) + static_cast<uint32_t>(b) * 4096u
+                        : smem_u32(sB + st * Plan::kBBytes) + static_cast<uint32_t>(b - kResPerA) * 4096u;
+  };
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + Plan::kMiscOffset);
   uint32_t *tmem_holder = misc;
   volatile uint32_t *abort_flag = misc + 1;
@@ -754,6 +775,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       mbar_init(bias_full_bar, kEpiWarps);  // lane 0 of each epilogue warp
       mbar_init(bias_free_bar, kEpiWarps);
     }
+    mbar_init(res_bar, 1);  // the producer's one arrive, plus the boxes' bytes
     *abort_flag = 0u;
     fence_mbar_init();
     if constexpr (!LSU) {
@@ -842,10 +864,45 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         }
       }
     }
+    // The last item's fp16 residual: once the final k-blocks no longer need the ring
+    // slots after them (their MMAs are done), those slots take the tile's residual rows,
+    // loaded while the last MMAs run.  The epilogue of the last tile, which nothing
+    // overlaps, then reads them from shared memory instead of waiting on DRAM.
+    int res_stages = 0;
+    if constexpr (kResSmem) {
+      const WorkItem wl = item(n_work > 0 ? n_work - 1 : 0);
+      if (ok && p.r_tma != 0 && n_work > 0 && wl.tail < 0) {
+        const int first = stage;
+        misc[2] = static_cast<uint32_t>(first);
+        const int y0 = wl.mb * kTileM + static_cast<int>(rank) * kBM;
+        for (int j = 0; j < kResBoxes && ok;) {
+          if (!mbar_wait_spin(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
+                              &g_device_error, 4096)) {
+            ok = false;
+            break;
+          }
+          const int nbox = kResBoxes - j < kResPerStage ? kResBoxes - j : kResPerStage;
+          mbar_expect_tx(res_bar, static_cast<uint32_t>(nbox) * 4096u);
+          for (int b = 0; b < nbox; ++b, ++j)
+            tma_load_2d(res_box(first, j), &tmR, res_bar,
+                        wl.nb * kTileN + (j % kResPieces) * 64, y0 + (j / kResPieces) * 32);
+          ++res_stages;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        mbar_arrive(res_bar);
+        // Every box issued has landed before this CTA's shared memory goes away, whatever
+        // the other roles do (no abort flag: the wait ends on the bytes or the limit).
+        mbar_wait(res_bar, 0, nullptr, p.limit_ns, kRoleProducer, &g_device_error);
+      }
+    }
     if (ok) {
       // Tail: wait until every slot has been released, so no commit-arrive is
-      // still on its way to this CTA's barriers when it exits.
-      for (int i = 0; i < STAGES; ++i) {
+      // still on its way to this CTA's barriers when it exits (the slots that took
+      // the residual were released before it went in).
+      for (int i = 0; i < STAGES - res_stages; ++i) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.limit_ns, kRoleProducer,
                        &g_device_error)) {
           ok = false;
@@ -1105,6 +1162,26 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
           add_bias_slice_32<kCPL>(bias, tcol + 32 * half, v);
       }
     };
+    // The residual pieces of the unit's last tile come from the ring (kResSmem, staged
+    // by the producer); every other piece is loaded from R by epi_prefetch.
+    bool r_smem = false;
+    uint32_t res_first = 0;
+    auto fetch_r = [&](int row, int col0, EpiIn<kPrefR> &in) {
+      if constexpr (kResSmem) {
+        if (r_smem) {
+          in.has_r = p.R != nullptr && col0 + 64 <= p.N && row < p.M;
+          if (in.has_r) {
+            const uint32_t box = res_box(static_cast<int>(res_first),
+                                         quarter * kResPieces + (col0 % kTileN) / 64) +
+                                 static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) in.r[c] = ld_shared_v4(box + static_cast<uint32_t>((c ^ (lane & 7)) * 16));
+          }
+          return;
+        }
+      }
+      epi_prefetch<kPrefR>(p, row, col0, in);
+    };
     auto pack = [&](float lo, float hi) {
       if constexpr (EK == kEpiBiasRelu)
         return pack_half2_relu(lo, hi);
@@ -1122,7 +1199,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) h[16 + j] = pack(vb[2 * j], vb[2 * j + 1]);
         if constexpr (kPrefR) {
-          if (next_col0 >= 0) epi_prefetch<kPrefR>(p, box_row0 + lane, next_col0, in);
+          if (next_col0 >= 0) fetch_r(box_row0 + lane, next_col0, in);
         }
         if (p.c_plain || (!p.n_aligned && col0 + kBoxCols > p.N)) {
           store_row_tail<true>(p, box_row0 + lane, col0, h);
@@ -1143,7 +1220,7 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
         epi32(in, bias, box_row0 + lane, col0, tcol, 0, va);
         epi32(in, bias, box_row0 + lane, col0, tcol, 1, vb);
         if constexpr (kPrefR) {
-          if (next_col0 >= 0) epi_prefetch<kPrefR>(p, box_row0 + lane, next_col0, in);
+          if (next_col0 >= 0) fetch_r(box_row0 + lane, next_col0, in);
         }
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -1296,9 +1373,10 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
       } else if constexpr (EK != kEpiNone) {
         if (p.bias != nullptr && w.nb * kTileN < p.N) load_bias_slice<kCPL>(p, w.nb * kTileN, lane, bias);
       }
+      r_smem = kResSmem && p.r_tma != 0 && k + 1 == n_work && w.tail < 0;
+      const int first_col = w.nb * kTileN + (KS > 1 ? kslice * Plan::kOwnCols : 0);
       if constexpr (kPrefR) {
-        const int first_col = w.nb * kTileN + (KS > 1 ? kslice * Plan::kOwnCols : 0);
-        if (w.tail < 0 && box_row0 < p.M && first_col < p.N)
+        if (!r_smem && w.tail < 0 && box_row0 < p.M && first_col < p.N)
           epi_prefetch<kPrefR>(p, box_row0 + lane, first_col, in);
       }
       // This wait spans the tile's whole main loop, so its limit grows with the
@@ -1310,6 +1388,13 @@ __global__ void __launch_bounds__(LSU ? kThreadsLsu : kThreads, 1)
                      &g_device_error))
         break;
       tc_fence_after_sync();
+      if constexpr (kResSmem) {
+        if (r_smem) {
+          if (!mbar_wait(res_bar, 0, abort_flag, p.limit_ns, kRoleEpilogue, &g_device_error)) break;
+          res_first = *reinterpret_cast<volatile uint32_t *>(misc + 2);
+          if (box_row0 < p.M && first_col < p.N) fetch_r(box_row0 + lane, first_col, in);
+        }
+      }
       if constexpr (KS > 1) {
         if (!ks_tile(w, box_row0, bias, in)) break;
       } else {

@@ -87,15 +87,15 @@ struct Variant {
   }
 
   static tlg_status launch(int units, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                           const CUtensorMap &tmC, const GemmParams &p, bool overlap_prev,
-                           cudaStream_t s) {
+                           const CUtensorMap &tmC, const CUtensorMap &tmR, const GemmParams &p,
+                           bool overlap_prev, cudaStream_t s) {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[2];
     fill_launch(&cfg, attr, s, overlap_prev);
     cfg.gridDim = dim3(static_cast<unsigned>(units * kClusterCtas), 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(
         &cfg, gemm_sm100_kernel<CG, BN, STAGES, OUT_F16, EK, NH, AT, BT, LSU, KS>, tmA, tmB, tmC,
-        p);
+        tmR, p);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return TLG_ERR_CUDA;
@@ -107,7 +107,7 @@ struct Variant {
 struct VariantFns {
   tlg_status (*units)(int, int, int *);
   tlg_status (*launch)(int, const CUtensorMap &, const CUtensorMap &, const CUtensorMap &,
-                       const GemmParams &, bool, cudaStream_t);
+                       const CUtensorMap &, const GemmParams &, bool, cudaStream_t);
 };
 
 
