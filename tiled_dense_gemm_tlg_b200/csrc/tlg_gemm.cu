@@ -118,15 +118,18 @@ struct KernelCfg {
 // TMA operands.  A CTA of such a cluster streams only its share of the
 // k-blocks, so a shape with few tiles keeps more SMs busy, and the wider tile
 // reads fewer operand bytes per FLOP than the 128 x 64 tile that would
-// otherwise spread it.  Their reduce_kb is the measured cost of the exchange,
-// in k-blocks of their tile (B200, one tile per cluster, fp32 C): about 1.3 us
-// for 32 KB per CTA each way, 2-5 us for 64-96 KB.  So they pay off only where
-// K is long next to M x N, not at 256^3 or 1024^3.
+// otherwise spread it.  Their reduce_kb is the cost of the exchange in k-blocks
+// of their tile (B200, one tile per cluster, fp32 C: about 1.3 us for 32 KB per
+// CTA each way, 2-5 us for 64-96 KB), fitted to forced runs of every tile on ten
+// long-K shapes from 256 x 256 x 4096 to 1536 x 1536 x 4096: the 128 x 256
+// clusters lost to the 128 x 128 tile, split or not, on all of them (512 x 768 x
+// 4096: 27.0 and 34.4 us against 22.0), so their exchange is charged 24 k-blocks.
+// So they pay off only where K is long next to M x N, not at 256^3 or 1024^3.
 constexpr KernelCfg kBuilt[] = {{1, 64, 8, 0.35, 0, true, 1, 0},   {1, 128, 6, 0.60, 0, false, 1, 0},
                                 {1, 256, 4, 0.90, 0, false, 1, 0},  {2, 128, 8, 0.60, 0, false, 1, 0},
                                 {2, 256, 6, 1.00, 0, true, 1, 0},   {2, 512, 4, 1.20, 19, false, 1, 0},
-                                {1, 128, 5, 0.60, 0, false, 2, 6.0}, {1, 256, 2, 0.90, 0, false, 2, 12.0},
-                                {1, 256, 2, 0.90, 0, false, 4, 12.0}};
+                                {1, 128, 5, 0.60, 0, false, 2, 6.0}, {1, 256, 2, 0.90, 0, false, 2, 24.0},
+                                {1, 256, 2, 0.90, 0, false, 4, 24.0}};
 constexpr int kNumBuilt = sizeof(kBuilt) / sizeof(kBuilt[0]);
 static_assert(kNumBuilt == kNumVariants, "one launcher table entry per built variant");
 
@@ -192,9 +195,20 @@ bool plan(int64_t tiles, int resident, int num_kb, int split, int cta_group, int
   s->tail_items = static_cast<int>(rem * split);
   s->workspace = split_workspace_bytes(s->tail_items, cta_group, block_n);
   // The slice runs first; its partial-sum traffic hides behind the next whole
-  // tile unless there is none, and then it costs about 2 + split k-blocks.
+  // tile unless there is none, and then it costs about 2 + split k-blocks.  The
+  // hiding fails for short tiles: with 16 k-blocks a split tail lost 4-11 %
+  // (8192 x 2048 x 1024, 12288 x 4096 x 1024, pair 256 tile) while at 64 it gains
+  // 4.5 %.  So each slice's fp32 partial, counted in k-blocks of operand bytes
+  // (the CTA's partial over its stage), is charged 0.3 of it, scaled by
+  // (16 / k-blocks)^2 up to 1.
   const double slice = static_cast<double>((num_kb + split - 1) / split);
-  s->cost = static_cast<double>(full) * num_kb + slice + (full > 0 ? 0.5 : 2.0 + split);
+  double fixup = 2.0 + split;
+  if (full > 0) {
+    const double partial_kb = (128.0 * block_n * 4.0) / (128.0 * kBK * 2.0 + kBK * (block_n / cta_group) * 2.0);
+    const double r = std::min(1.0, 16.0 / num_kb);
+    fixup = 0.5 + 0.3 * split * partial_kb * r * r;
+  }
+  s->cost = static_cast<double>(full) * num_kb + slice + fixup;
   return true;
 }
 
