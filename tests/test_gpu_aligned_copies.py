@@ -127,10 +127,11 @@ def test_size_query_for_aligned_operands_is_the_split_scratch(tlg):
 
 def test_size_query_bytes_hold_the_split_and_the_copy(tlg):
     # 108 pair tiles (3072 x 2304): one whole wave, then a tail the automatic choice cuts in two
-    # along K when the workspace holds the slices' partial sums.  Only A needs a copy.  With
-    # exactly the size query's bytes the call must take the same schedule as the query: the
-    # split scratch first, then A's aligned copy, ending at the workspace's last byte.
-    M, N, K = 3072, 2304, 512
+    # along K when the workspace holds the slices' partial sums (K = 2048: 32 k-blocks, long
+    # enough that the model keeps the split).  Only A needs a copy.  With exactly the size
+    # query's bytes the call must take the same schedule as the query: the split scratch
+    # first, then A's aligned copy, ending at the workspace's last byte.
+    M, N, K = 3072, 2304, 2048
     A, B, bias = wl.make_operands(M, N, K, "uniform", bias=True, seed=406)
     lib = tlg.raw_library()
     ra = Raw(A, M, K, K + 1, torch.float16, 0)
@@ -139,7 +140,7 @@ def test_size_query_bytes_hold_the_split_and_the_copy(tlg):
     rcq = lib.tlg_gemm_workspace_size_op(M, N, K, 0, ra.ptr(), ra.ld, 0, Bd.data_ptr(), N, C.data_ptr(), N,
                                          tlg.TLG_OUT_F16, None, ctypes.byref(full))
     assert rcq == 0, tlg.tlg_status_string(rcq)
-    a_copy = M * K * 2  # rows of 1024 bytes: already 16- and 256-byte multiples
+    a_copy = M * K * 2  # rows of 4096 bytes: already 16- and 256-byte multiples
     split_ws = tlg.tlg_gemm_workspace_size(M, N, K, "f16", True)
     assert split_ws > 4096, "the automatic choice no longer splits this shape"
     assert full.value == (split_ws + 255) // 256 * 256 + a_copy
