@@ -396,6 +396,8 @@ def main(argv=None):
     ap.add_argument("--config", default=None, help="JSON tlg_config override (tuning sweeps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-library", action="store_true",
+                    help="skip the same-box torch/cuBLAS comparison timing")
     ap.add_argument("--layout", default="NN", choices=["NN", "NT", "TN", "TT"],
                     help="op(A), op(B): T = that operand is stored transposed (tlg_gemm_op)")
     ap.add_argument("--sustained-s", type=float, default=3.0,
@@ -575,6 +577,54 @@ def main(argv=None):
         plain = {"call": plain_name, "value": w.flops * args.steps * world / (plain_ms * 1e-3) / 1e12,
                  "unit": UNIT, "ms_per_step": plain_ms / args.steps}
 
+    # ---- cuBLAS on the same box, for comparison only (never part of `value`): torch.mm of the
+    # same fp16 operands into a C of the workload's type, timed the same way (L2 flushed before
+    # every call, CUDA events on the same stream); with a bias, also torch's own composition of
+    # the workload's epilogue (addmm, the activation, the residual add: separate kernels).
+    library = None
+    if not args.no_library and world == 1 and not use_op:
+        import torch.nn.functional as F
+
+        Cl = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+        out32 = w.out == "f32"  # fp16 operands into an fp32 C (torch's mm with out_dtype)
+        if out32:
+            try:
+                torch.mm(dA[:8, :8], dB[:8, :8], out_dtype=torch.float32)
+            except Exception:
+                out32 = False
+        act = w.act if fused else ("relu" if dbias is not None else None)
+        act_fn = {"relu": F.relu, "gelu": F.gelu, "silu": F.silu,
+                  "gelu_tanh": lambda x: F.gelu(x, approximate="tanh"), "none": lambda x: x}
+
+        def lib_mm():
+            with torch.cuda.stream(stream):
+                if out32:
+                    torch.mm(dA, dB, out_dtype=torch.float32)
+                else:
+                    torch.mm(dA, dB, out=Cl)
+
+        def lib_epi():
+            with torch.cuda.stream(stream):
+                x = act_fn[act](torch.addmm(dbias, dA, dB))
+                if dR is not None:
+                    x = x + dR
+
+        def lib_time(fn, call):
+            for _ in range(args.warmup):
+                flush.fill_(1.0)
+                fn()
+            torch.cuda.synchronize(dev)
+            ms = sum(timed(fn, args.steps))
+            return {"call": call, "value": w.flops * args.steps / (ms * 1e-3) / 1e12, "unit": UNIT,
+                    "ms_per_step": ms / args.steps}
+
+        library = lib_time(lib_mm, "torch.mm (cuBLAS), " + ("fp32 C (out_dtype)" if out32 else "fp16 C") +
+                           ", no epilogue")
+        if dbias is not None and dA.dtype == torch.float16:
+            library["with_epilogue"] = lib_time(
+                lib_epi, f"torch.addmm + {act}" + (" + residual" if dR is not None else "") +
+                f", {'fp16' if w.out == 'f16' else 'fp16 (the workload writes fp32)'} C, separate kernels")
+
     max_ms = max_over_ranks(gemm_ms, world)
     total_flops = w.flops * args.steps * world
     value = job_throughput(w.flops, args.steps, world, max_ms)
@@ -729,6 +779,7 @@ def main(argv=None):
                                       else "plain loads/stores") + " (row strides not 16-byte multiples)"
                                      if (args.ld_pad * 2) % 16 else "TMA")),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "plain_entry_point": plain,
+        "library_same_box": library,
         "sustained": sustained,
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clk,

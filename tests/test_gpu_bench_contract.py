@@ -32,5 +32,7 @@ def test_default_bench_line_has_the_contract_keys():
     assert e["value"] > 0 and e["h2d_bytes_per_step"] == 2 * (2 * 4096 * 4096) + 2 * 4096
     assert e["d2h_bytes_per_step"] == 2 * 4096 * 4096
     assert d["gpu_launches"] == 3  # one GEMM per timed step
+    lib = d["library_same_box"]  # cuBLAS timed the same way on the same box, for comparison
+    assert lib["value"] > 0 and "torch.mm" in lib["call"] and lib["with_epilogue"]["value"] > 0
     if d["clocks"] is not None:
         assert d["clocks"]["sm_mhz"] > 0 and isinstance(d["clocks"]["reasons"], list)
