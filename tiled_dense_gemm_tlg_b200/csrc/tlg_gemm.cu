@@ -194,8 +194,9 @@ bool plan(int64_t tiles, int resident, int num_kb, int split, int cta_group, int
   s->split = split;
   s->tail_items = static_cast<int>(rem * split);
   s->workspace = split_workspace_bytes(s->tail_items, cta_group, block_n);
-  // The slice runs first; its partial-sum traffic hides behind the next whole
-  // tile unless there is none, and then it costs about 2 + split k-blocks.  The
+  // A whole tile follows the slice (see work_item), so its partial-sum traffic
+  // hides behind that tile's main loop unless there is none, and then it costs
+  // about 2 + split k-blocks.  The
   // hiding fails for short tiles: with 16 k-blocks a split tail lost 4-11 %
   // (8192 x 2048 x 1024, 12288 x 4096 x 1024, pair 256 tile) while at 64 it gains
   // 4.5 %.  So each slice's fp32 partial, counted in k-blocks of operand bytes
