@@ -157,3 +157,26 @@ def test_workspace_size_op_host_checks(lib_path):
     assert lib.tlg_gemm_workspace_size_op(8, 8, 8, 0, A, 7, 0, A, 8, A * 2, 8, 1, None, ctypes.byref(n)) == tlg.TLG_ERR_INVALID_ARG
     assert lib.tlg_gemm_workspace_size_op(0, 8, 8, 0, None, 8, 0, None, 8, None, 8, 1, None, ctypes.byref(n)) == tlg.TLG_OK
     assert n.value == 0
+
+
+def test_gelu_tail_coefficients_are_the_fits(lib_path):
+    # The kernel's GELU tail polynomials (one per type of C) are the ones the fit script
+    # beside the kernel prints, to the last float32 digit, and their degrees match.
+    import importlib.util
+
+    import numpy as np
+
+    csrc = os.path.join(ROOT, "tiled_dense_gemm_tlg_b200", "csrc")
+    spec = importlib.util.spec_from_file_location("fit_gelu_tail", os.path.join(csrc, "fit_gelu_tail.py"))
+    fit = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(fit)
+    src = open(os.path.join(csrc, "tlg_gemm_kernel.cuh")).read()
+    body = src[src.index("gelu_tail_coef(int k)"):src.index("kGeluTailDegree")]
+    arrays = re.findall(r"constexpr float c\[(\d+)\] = \{([^}]*)\}", body)
+    assert len(arrays) == 2
+    for (n, vals), out in zip(arrays, ("f16", "f32")):  # the fp16 fit is written first
+        kernel = np.array([float(v.strip().rstrip("f")) for v in vals.split(",")], dtype=np.float32)
+        assert int(n) == fit.DEGREE[out] + 1 == kernel.size
+        assert np.array_equal(kernel, fit.fit(out)), out
+    degrees = re.search(r"kGeluTailDegree = F16 \? (\d+) : (\d+);", src)
+    assert (int(degrees.group(1)), int(degrees.group(2))) == (fit.DEGREE["f16"], fit.DEGREE["f32"])

@@ -237,6 +237,33 @@ def test_gelu_matches_exact_form_pointwise(tlg):
     assert err.max() <= 1e-6 * (1 + np.abs(ref).max()), err.max()
 
 
+def _ulp_f16(v: np.ndarray) -> np.ndarray:
+    """The fp16 unit in the last place at |v| (the subnormal spacing below 2^-14)."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -14)))
+    return 2.0 ** (e - 10)
+
+
+def test_gelu_fp16_output_within_a_fraction_of_an_ulp(tlg):
+    # A = I: C = gelu(B) rounded to fp16, for every fp16 value B in [-16, 16] (fp16
+    # subnormals included).  Before the rounding the kernel's GELU is within 0.15 fp16
+    # units in the last place of the exact form, so each stored result lies within
+    # 0.65 units of the fp64 oracle (a correct rounding alone allows 0.5).
+    h = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16).view(torch.float16)
+    h = h[torch.isfinite(h) & (h.abs() <= 16)]
+    N = 640
+    assert h.numel() <= 64 * N
+    x = torch.zeros(64 * N, dtype=torch.float16)
+    x[: h.numel()] = h
+    x = x.reshape(64, N)
+    A = torch.eye(64, dtype=torch.float16)
+    got = tlg.tlg_gemm_fused(A.cuda(), x.cuda(), activation="gelu", out="f16")
+    torch.cuda.synchronize()
+    ref = oracle.gemm_fused(A, x, act="gelu")
+    err_ulp = np.abs(got.double().cpu().numpy() - ref) / _ulp_f16(ref)
+    worst = np.unravel_index(int(np.argmax(err_ulp)), err_ulp.shape)
+    assert err_ulp.max() <= 0.65, (err_ulp.max(), float(x[worst]))
+
+
 def test_argument_errors_on_device(tlg):
     lib = tlg.raw_library()
     A = torch.ones((64, 64), dtype=torch.float16, device="cuda")

@@ -274,49 +274,75 @@ __device__ __forceinline__ void add_half2_to(float &x0, float &x1, uint32_t w) {
 //   x Phi(x) = max(x, 0) - a q
 // (x (1 - q) for x >= 0, -|x| q for x < 0; beyond |x| = 6, q < 1e-9 and a q
 // < 6e-9): one fused multiply-add, no select, and q is computed directly, so
-// the negative tail has no cancellation.  q = 2^g(a) with g a degree-6
-// polynomial fitted to log2 Phi(-a) on [0, 6], its error weighted by what it
-// costs in GELU (a Phi(-a) ln 2) and made near-minimax by Lawson's
+// the negative tail has no cancellation.  q = 2^g(a) with g a polynomial
+// fitted to log2 Phi(-a) on [0, 6] and made near-minimax by Lawson's
 // reweighted least squares (fit_gelu_tail.py beside this file prints the
-// coefficients; GELU error below 3e-7 on [-8, 8] in fp32).  One exp2 and no
-// reciprocal: the special-function unit the epilogue shares with its SM
-// partition is its scarcest resource.  min.NaN keeps a NaN input NaN.
-constexpr float kGeluG0 = -0.999993086f, kGeluG1 = -1.15120173f, kGeluG2 = -0.458770931f,
-                kGeluG3 = -0.0534121692f, kGeluG4 = 0.00808076002f, kGeluG5 = -0.000769232807f,
-                kGeluG6 = 3.30943076e-05f;
-
-__device__ __forceinline__ float gelu_tail_arg(float x) {  // min(|x|, 6), NaN stays NaN
-  float a;
-  asm("min.NaN.f32 %0, %1, %2;" : "=f"(a) : "f"(fabsf(x)), "f"(6.0f));
-  return a;
+// coefficients and the errors).  Two fits, by the type of C:
+//  - fp32 C: degree 6, the error weighted by what it costs in GELU
+//    (a Phi(-a) ln 2): GELU error below 3e-7 on [-8, 8];
+//  - fp16 C: degree 5, the error weighted in fp16 units in the last place
+//    of a Phi(-a): at most 0.14 of a unit before the rounding to fp16, so
+//    every fp16 result lies within 0.64 units of the exact GELU.
+// One exp2 and no reciprocal.  The epilogue's instruction count is what the
+// main loop running beside it feels, so the form is written for the fewest:
+// the polynomial runs in na = -a = max.NaN(-|x|, -6) with the odd
+// coefficients negated (sum c_k a^k = sum (-1)^k c_k na^k).  Each Horner step
+// then yields exactly the negation of the step in a (round to nearest is
+// symmetric), so g has the same bits, and -a q + max(x, 0) is one packed
+// fused multiply-add for two values.  max.NaN keeps a NaN input NaN.
+template <bool F16>
+__device__ __forceinline__ constexpr float gelu_tail_coef(int k) {  // c_k, lowest degree first
+  if constexpr (F16) {
+    constexpr float c[6] = {-1.00010169f, -1.14941466f, -0.463673383f, -0.0485566817f,
+                            0.00592234265f, -0.000330398412f};
+    return c[k];
+  } else {
+    constexpr float c[7] = {-0.999993086f,  -1.15120173f,     -0.458770931f, -0.0534121692f,
+                            0.00808076002f, -0.000769232807f, 3.30943076e-05f};
+    return c[k];
+  }
 }
 
+template <bool F16>
+constexpr int kGeluTailDegree = F16 ? 5 : 6;
+
+// The coefficient of na^k.
+template <bool F16>
+__device__ __forceinline__ constexpr float gelu_tail_coef_neg(int k) {
+  return (k & 1) ? -gelu_tail_coef<F16>(k) : gelu_tail_coef<F16>(k);
+}
+
+__device__ __forceinline__ float gelu_tail_narg(float x) {  // -min(|x|, 6), NaN stays NaN
+  float na;
+  asm("{\n\t.reg .f32 t;\n\tabs.f32 t, %1;\n\tneg.f32 t, t;\n\tmax.NaN.f32 %0, t, %2;\n\t}"
+      : "=f"(na)
+      : "f"(x), "f"(-6.0f));
+  return na;
+}
+
+template <bool F16>
 __device__ __forceinline__ float gelu_erf(float x) {
-  const float a = gelu_tail_arg(x);
-  float g = fmaf(kGeluG6, a, kGeluG5);
-  g = fmaf(g, a, kGeluG4);
-  g = fmaf(g, a, kGeluG3);
-  g = fmaf(g, a, kGeluG2);
-  g = fmaf(g, a, kGeluG1);
-  g = fmaf(g, a, kGeluG0);
-  return fmaf(-a, ex2_approx(g), fmaxf(x, 0.0f));  // q = 2^g = Phi(-a)
+  constexpr int D = kGeluTailDegree<F16>;
+  const float na = gelu_tail_narg(x);
+  float g = gelu_tail_coef_neg<F16>(D);
+#pragma unroll
+  for (int k = D - 1; k >= 0; --k) g = fmaf(g, na, gelu_tail_coef_neg<F16>(k));
+  return fmaf(na, ex2_approx(g), fmaxf(x, 0.0f));  // 2^g = q = Phi(-a)
 }
 
-// gelu_erf on two values, the polynomial with the packed instructions: the same
-// operations in the same order, so the same bits.
+// gelu_erf on two values with the packed instructions: the same operations in
+// the same order, so the same bits.
+template <bool F16>
 __device__ __forceinline__ void gelu_erf_2(float &x0, float &x1) {
-  const float a0 = gelu_tail_arg(x0), a1 = gelu_tail_arg(x1);
-  const uint64_t a = f2_pack(a0, a1);
-  uint64_t g = f2_fma(f2_splat(kGeluG6), a, f2_splat(kGeluG5));
-  g = f2_fma(g, a, f2_splat(kGeluG4));
-  g = f2_fma(g, a, f2_splat(kGeluG3));
-  g = f2_fma(g, a, f2_splat(kGeluG2));
-  g = f2_fma(g, a, f2_splat(kGeluG1));
-  g = f2_fma(g, a, f2_splat(kGeluG0));
+  constexpr int D = kGeluTailDegree<F16>;
+  const uint64_t na = f2_pack(gelu_tail_narg(x0), gelu_tail_narg(x1));
+  uint64_t g = f2_splat(gelu_tail_coef_neg<F16>(D));
+#pragma unroll
+  for (int k = D - 1; k >= 0; --k) g = f2_fma(g, na, f2_splat(gelu_tail_coef_neg<F16>(k)));
   float g0, g1;
   f2_unpack(g, g0, g1);
-  x0 = fmaf(-a0, ex2_approx(g0), fmaxf(x0, 0.0f));
-  x1 = fmaf(-a1, ex2_approx(g1), fmaxf(x1, 0.0f));
+  const uint64_t m = f2_pack(fmaxf(x0, 0.0f), fmaxf(x1, 0.0f));
+  f2_unpack(f2_fma(na, f2_pack(ex2_approx(g0), ex2_approx(g1)), m), x0, x1);
 }
 
 // SiLU and the tanh form of GELU are both x * sigmoid(c1 x + c3 x^3):
@@ -351,22 +377,24 @@ __device__ __forceinline__ void sigmoid_form_apply_2(SigmoidForm f, float &x0, f
   f2_unpack(f2_mul(x, f2_pack(rcp_approx(d0), rcp_approx(d1))), x0, x1);
 }
 
+template <bool F16>
 __device__ __forceinline__ float activate(int act, float x) {
   if (act == kActRelu) return fmaxf(x, 0.0f);
-  if (act == kActGelu) return gelu_erf(x);
+  if (act == kActGelu) return gelu_erf<F16>(x);
   if (act == kActSilu || act == kActGeluTanh) return sigmoid_form_apply(sigmoid_form(act), x);
   return x;
 }
 
 // The activation over 32 values; `act` is the same for every thread, so the
-// branch does not diverge.
+// branch does not diverge.  F16: the result is rounded to fp16 (GELU's fit).
+template <bool F16>
 __device__ __forceinline__ void activate_32(int act, float (&v)[32]) {
   if (act == kActRelu) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
   } else if (act == kActGelu) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) gelu_erf_2(v[j], v[j + 1]);
+    for (int j = 0; j < 32; j += 2) gelu_erf_2<F16>(v[j], v[j + 1]);
   } else if (act == kActSilu || act == kActGeluTanh) {
     const SigmoidForm f = sigmoid_form(act);
 #pragma unroll
@@ -530,7 +558,7 @@ __device__ __forceinline__ void epi_apply_32(const GemmParams &p, const EpiIn<ON
     else
       add_bias_slice_32<CPL>(bias, tcol + 32 * half, v);
   }
-  activate_32(p.act, v);
+  activate_32<OUT_F16>(p.act, v);
   if (p.R != nullptr) {
     if (ON && in.has_r) {
 #pragma unroll
@@ -1543,7 +1571,7 @@ __global__ void fill_empty_k_kernel(void *C, int64_t ldc, const __half *bias, in
     float v = 0.0f;
     if constexpr (EPI) {
       if (bias != nullptr) v = __half2float(bias[c]);
-      v = activate(act, v);
+      v = activate<OUT_F16>(act, v);
       if (R != nullptr)
         v += OUT_F16 ? __half2float(static_cast<const __half *>(R)[r * ldr + c])
                      : static_cast<const float *>(R)[r * ldr + c];
