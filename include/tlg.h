@@ -281,7 +281,12 @@ typedef enum tlg_activation {
  *   C[i][j] = act(acc[i][j] + bias[j]) + residual[i][j]
  *
  * acc is the fp32 accumulator of op(A) . op(B); everything is computed in
- * fp32 and rounded once to C's type at the store.
+ * fp32 and rounded once to C's type at the store.  Activation accuracy:
+ * GELU is within 3e-7 of the exact form for an fp32 C; for an fp16 C its
+ * fp32 value is within 0.15 fp16 units in the last place, so the stored
+ * result is within 0.65 units.  SiLU and the tanh form use the hardware
+ * exp2 and reciprocal approximations: on [-12, 12] their error stays below
+ * 2e-6 times (1 + the largest |value|).
  *   bias       : N fp16 values (device memory), or NULL for none
  *   activation : a tlg_activation
  *   residual   : M x N row-major in C's type (fp16 for TLG_OUT_F16, fp32 for
