@@ -262,6 +262,15 @@ def test_gelu_fp16_output_within_a_fraction_of_an_ulp(tlg):
     err_ulp = np.abs(got.double().cpu().numpy() - ref) / _ulp_f16(ref)
     worst = np.unravel_index(int(np.argmax(err_ulp)), err_ulp.shape)
     assert err_ulp.max() <= 0.65, (err_ulp.max(), float(x[worst]))
+    # With a bias the activation's input x + bias is an fp32 value between the fp16 points;
+    # the bound is the same (the fit holds on every fp32 input, not only fp16 ones).
+    bias = (torch.arange(N, dtype=torch.float32) % 7 - 3).mul(0.1).half()
+    got = tlg.tlg_gemm_fused(A.cuda(), x.cuda(), bias=bias.cuda(), activation="gelu", out="f16")
+    torch.cuda.synchronize()
+    ref = oracle.gemm_fused(A, x, bias=bias, act="gelu")
+    err_ulp = np.abs(got.double().cpu().numpy() - ref) / _ulp_f16(ref)
+    worst = np.unravel_index(int(np.argmax(err_ulp)), err_ulp.shape)
+    assert err_ulp.max() <= 0.65, (err_ulp.max(), float(x[worst]), float(bias[worst[1]]))
 
 
 def test_argument_errors_on_device(tlg):
