@@ -221,9 +221,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // Packed fp32 pairs.  sm_100's add/mul/fma .f32x2 do two fp32 operations
 // in one instruction, each rounded exactly as its scalar form, so a pair of
-// columns costs the issue slot of one: the epilogue's arithmetic competes with
-// the producer and MMA warps for the SM's issue slots.  The pair sits in one
-// 64-bit register (the even column in the low word).
+// columns costs the issue slot of one (the epilogue warps share each SM
+// sub-partition's issue slots with the producer and MMA warps).  The pair
+// sits in one 64-bit register (the even column in the low word).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
